@@ -1,0 +1,226 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts block.
+ *
+ * The block, as the pages define it:
+ *   route    sigmoid router with a selection-only expert bias and normalised
+ *            top-k: s = sigmoid(x . W_router^T); the k experts with the
+ *            largest s + bias are picked; w_j = s_j / (sum_j s_j + eps) * scale.
+ *            (TileGym PR #187 "[E2E Model Support] Add TileGym kernel
+ *            integration for LFM2 MoE", section "Weight layout and routing";
+ *            TensorFold pull #1492, sections "What" and "Verification".)
+ *   plan     the grouped expert plan: per-expert counts, offsets and the
+ *            permutation of routed pairs (TensorFold issue #548, "Zig CUDA
+ *            ports: shared layers below lanes.Backend ...", the shared
+ *            grouped-MoE layer and its routing plan).
+ *   experts  grouped expert GEMMs: gate_up (E, 2I, H) gate-first with a SwiGLU
+ *            epilogue, or the non-gated up (E, I, H) -> relu^2; then down
+ *            (E, H, I) whose output is weighted by w and summed into the
+ *            token's row (TileGym PR #187 "Weight layout and routing";
+ *            vllm.cpp PR #684 "W2 (MODEL-NEMOTRON-H): the non-gated relu^2 MoE
+ *            expert", section "The seam decision").
+ *   combine  y = out_scale * sum_j w_j * expert_j(x): the output scale
+ *            multiplies the finished sum once (vllm.cpp PR #684, "The finding
+ *            that justifies the row").
+ *
+ * Conventions for every entry point
+ *   - Pointers named x, logits, w_router, expert_bias, topk_*, plan arrays,
+ *     weights, y and ws are DEVICE pointers (the caller owns the memory; the
+ *     library allocates nothing on these paths).  moe_forward_host is the one
+ *     exception and says so.
+ *   - Layouts are dense row-major.  bf16 tensors are IEEE bfloat16 bit
+ *     patterns (uint16).  Indices are int32.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  No entry point synchronises the host, except
+ *     moe_device_error and moe_forward_host.
+ *   - A non-OK status comes from host-side validation before anything is
+ *     launched (MOE_ERR_NULL/SHAPE/ALIGN/UNSUPPORTED/WORKSPACE) or from a
+ *     failed launch (MOE_ERR_CUDA).  moe_last_error() then returns a message
+ *     for the calling thread.  Validation failures enqueue nothing.
+ *   - Kernels never trap.  A device-side check that fails (an expert id out
+ *     of range, a bounded wait that expired) writes a code to the library's
+ *     device error word and the kernel returns; moe_device_error() reads it.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_NULL = 1,        /* a required pointer is NULL */
+    MOE_ERR_SHAPE = 2,       /* a size is out of range (see each call) */
+    MOE_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+    MOE_ERR_UNSUPPORTED = 4, /* an enum value or combination this build does not run */
+    MOE_ERR_WORKSPACE = 5,   /* ws is NULL or smaller than moe_workspace_bytes() */
+    MOE_ERR_CUDA = 6,        /* a CUDA runtime call or launch failed */
+    MOE_ERR_DEVICE = 7       /* moe_device_error found a device-side error code */
+} moe_status;
+
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act;
+typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1 } moe_wfmt;
+
+/* Which expert kernels moe_experts / moe_forward use (process-wide). */
+typedef enum {
+    MOE_DISPATCH_AUTO = 0, /* grouped GEMV when T <= 64, tcgen05 grouped GEMM above */
+    MOE_DISPATCH_GEMV = 1, /* always the weight-streaming grouped GEMV */
+    MOE_DISPATCH_GEMM = 2  /* always the tcgen05 grouped GEMM */
+} moe_dispatch;
+
+/* Problem sizes.  T tokens, H hidden, E experts, k picks per token, I expert
+ * intermediate width.  P = T * k routed pairs.
+ * Limits: 0 <= T, T * k < 2^31; H % 64 == 0 and 64 <= H <= 16384;
+ *         I % 64 == 0 and 64 <= I <= 16384; 1 <= E <= 256; 1 <= k <= min(E, 32). */
+typedef struct {
+    int32_t T, H, E, k, I;
+} moe_dims;
+
+/* Expert weights (device pointers).
+ *   fmt = MOE_W_BF16:
+ *     act SWIGLU: w1 = gate_up (E, 2I, H) bf16, rows [0, I) gate, [I, 2I) up;
+ *     act RELU2:  w1 = up (E, I, H) bf16;
+ *     w2 = down (E, H, I) bf16.  *_scale and *_bias are unused (may be NULL).
+ *   fmt = MOE_W_AFFINE4_G64 (MLX-style affine 4-bit, group 64 along K):
+ *     w1 = codes (E, N1, H/8) uint32 with N1 = 2I (SWIGLU) or I (RELU2),
+ *     w1_scale, w1_bias = (E, N1, H/64) bf16;
+ *     w2 = codes (E, H, I/8) uint32, w2_scale, w2_bias = (E, H, I/64) bf16.
+ *     A uint32 holds 8 consecutive k, the low nibble first; the weight is
+ *     scale * q + bias (TensorFold pull #1492, "What": Affine4 experts). */
+typedef struct {
+    int32_t fmt; /* moe_wfmt */
+    int32_t act; /* moe_act */
+    const void* w1;
+    const void* w1_scale;
+    const void* w1_bias;
+    const void* w2;
+    const void* w2_scale;
+    const void* w2_bias;
+} moe_experts_w;
+
+/* The routing plan (device arrays the caller allocates).
+ *   counts  [E]    pairs routed to each expert
+ *   offsets [E+1]  exclusive scan of counts
+ *   perm    [P]    pair ids p = t*k + j sorted stably by (expert, p)
+ *   inv     [P]    inv[p] = position of pair p in perm
+ *   tiles   [E+1]  exclusive scan of ceil(counts / MOE_TILE_M): the grouped
+ *                  GEMM's M-tile table (tiles[E] = number of M-tiles) */
+typedef struct {
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* perm;
+    int32_t* inv;
+    int32_t* tiles;
+} moe_plan_t;
+
+#define MOE_TILE_M 128
+
+/* Byte offsets of the regions inside the workspace (for inspection/tests). */
+typedef struct {
+    size_t y_acc;   /* fp32 (T, H): the unscaled routed sum */
+    size_t h;       /* bf16 (P, I): activations in plan order */
+    size_t xs;      /* bf16 (P, H): x rows gathered in plan order (GEMM path) */
+    size_t scratch; /* plan and scheduler scratch */
+    size_t total;   /* == moe_workspace_bytes() */
+} moe_ws_layout;
+
+/* Bytes of device workspace moe_plan / moe_experts / moe_forward need for
+ * these sizes and weight format (0 on invalid sizes).  256-byte aligned
+ * regions; ws itself must be 256-byte aligned. */
+MOE_API size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt);
+MOE_API moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* out);
+
+/* Router.  Exactly one of x (bf16 (T, H)) or logits (fp32 (T, E)) is given;
+ * with x, w_router (fp32 (E, H)) is required and the logits are computed in
+ * fp32 with a fixed summation order (a token's result never depends on T).
+ * expert_bias (fp32 (E)) may be NULL (no bias).  Writes topk_idx (T, k) int32
+ * in rank order (descending s + bias, ties to the lower id, NaN last; an
+ * all-NaN row picks 0..k-1) and topk_w (T, k) fp32 = s / (sum s + eps) * scale.
+ * A row whose logits are all NaN gets NaN weights. */
+MOE_API moe_status moe_route(const void* x, const float* logits, const float* w_router,
+                     const float* expert_bias, const moe_dims* d, float eps, float scale,
+                     int32_t* topk_idx, float* topk_w, moe_stream_t stream);
+
+/* Plan of topk_idx (T, k) int32 (values must lie in [0, E); a value outside
+ * sets device error code 1 and is counted nowhere).  Fills every array of
+ * *plan.  Uses the scratch region of ws. */
+MOE_API moe_status moe_plan(const int32_t* topk_idx, const moe_dims* d, const moe_plan_t* plan, void* ws,
+                    size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped experts + combine: y (T, H) bf16 = bf16_rn(out_scale * y_acc) where
+ * y_acc[t] = sum_j topk_w[t, j] * down_e(act(up_e(x[t]))) in fp32, e = the
+ * pair's expert.  The activation is rounded once to bf16 (stored in ws.h);
+ * y_acc is kept in ws.y_acc.  Rows of y for tokens with no pairs are 0. */
+MOE_API moe_status moe_experts(const void* x, const moe_plan_t* plan, const float* topk_w,
+                       const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* route -> plan -> experts -> combine in one call (same arguments as the three
+ * calls; logits may be NULL to route from x). */
+MOE_API moe_status moe_forward(const void* x, const float* logits, const float* w_router,
+                       const float* expert_bias, const moe_dims* d, float eps, float router_scale,
+                       float out_scale, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
+                       const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
+                       moe_stream_t stream);
+
+/* moe_forward with HOST buffers for the token rows: x_host (T, H) bf16 is
+ * copied to x_dev, the block runs, and y_dev is copied back to y_host (T, H)
+ * bf16, all on `stream`; the call then synchronises `stream`.  x_host/y_host
+ * should be pinned for the copies to be asynchronous.  Everything else is as
+ * moe_forward (device pointers). */
+MOE_API moe_status moe_forward_host(const void* x_host, void* x_dev, const float* w_router,
+                            const float* expert_bias, const moe_dims* d, float eps,
+                            float router_scale, float out_scale, const moe_experts_w* W,
+                            int32_t* topk_idx, float* topk_w, const moe_plan_t* plan, void* y_dev,
+                            void* y_host, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Stages of the block, for moe_profile_hook. */
+typedef enum {
+    MOE_STAGE_ROUTE = 0,   /* the router kernel(s): logits + selection (+ plan for T <= 32) */
+    MOE_STAGE_PLAN = 1,    /* the plan kernel (fused into the router for T <= 32) */
+    MOE_STAGE_UP = 2,      /* the expert up-projection + activation kernel */
+    MOE_STAGE_DOWN = 3,    /* the expert down-projection + weighted scatter kernel */
+    MOE_STAGE_FINAL = 4    /* the output scale + bf16 rounding kernel */
+} moe_stage;
+
+/* One-shot timing hook for the calling thread: the next moe_forward /
+ * moe_experts call on this thread records ev_begin (a cudaEvent_t) on its
+ * stream just before launching `stage`'s kernel and ev_end just after, then
+ * forgets the hook.  Pass NULL events to clear it.  Works under stream
+ * capture (the records become event nodes). */
+MOE_API moe_status moe_profile_hook(void* ev_begin, void* ev_end, int32_t stage);
+
+/* Number of kernels the calling thread's last successful moe_* call launched. */
+MOE_API int32_t moe_last_launch_count(void);
+
+/* Process-wide choice of expert kernels (moe_dispatch); returns the old one. */
+MOE_API int32_t moe_set_dispatch(int32_t mode);
+
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  *code = 0 when no kernel reported an error.  Codes:
+ * 1 expert id out of range in moe_plan; 2 a bounded pipeline wait expired in
+ * a grouped GEMM kernel.  Returns MOE_ERR_DEVICE when *code != 0. */
+MOE_API moe_status moe_device_error(int32_t* code, moe_stream_t stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Library version string. */
+MOE_API const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,83 @@
+// Host-side interfaces between the C-ABI layer (moe_api.cu) and the kernel
+// files.  Plain structs of device pointers and sizes; nothing here allocates.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct RouteArgs {
+    const uint16_t* x;       // (T, H) bf16, or null when logits are given
+    const float* logits;     // (T, E) fp32, or null
+    const float* w_router;   // (E, H) fp32
+    const float* bias;       // (E) fp32 or null
+    float* l_scratch;        // (T, E) fp32 scratch for the small-T logits pass
+    int T, H, E, k;
+    float eps, scale;
+    int32_t* idx;            // (T, k)
+    float* w;                // (T, k)
+    // optional fused plan (single-CTA select path only)
+    int32_t *counts, *offsets, *perm, *inv, *tiles;
+    // optional zeroing of the fp32 accumulator (forward path)
+    float* zero_ptr;
+    size_t zero_count;       // floats
+    int* err;
+};
+
+struct PlanArgs {
+    const int32_t* idx;
+    int P, E, k;
+    int32_t *counts, *offsets, *perm, *inv, *tiles;
+    int* err;
+};
+
+struct ExpertArgs {
+    const uint16_t* x;       // (T, H) bf16
+    const float* topk_w;     // (T, k)
+    const int32_t* counts;
+    const int32_t* offsets;
+    const int32_t* perm;
+    const int32_t* tiles;
+    int T, H, E, k, I;
+    int act;                 // 0 swiglu, 1 relu2
+    int fmt;                 // 0 bf16, 1 affine4
+    const void* w1;
+    const uint16_t* w1_scale;
+    const uint16_t* w1_bias;
+    const void* w2;
+    const uint16_t* w2_scale;
+    const uint16_t* w2_bias;
+    uint16_t* h;             // (P, I) bf16 in plan order
+    uint16_t* xs;            // (P, H) bf16 gathered rows (GEMM path)
+    float* y_acc;            // (T, H) fp32
+    uint16_t* y;             // (T, H) bf16
+    float out_scale;
+    int* err;
+};
+
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;
+    int* err_word;           // device address of this device's error word
+};
+
+const DeviceInfo& device_info();   // of the current device (cached)
+
+// Launchers: return the first CUDA error, cudaSuccess otherwise.
+// launch_route sets *n_launched to the number of kernels it enqueued.
+cudaError_t launch_route(const RouteArgs& a, bool fuse_plan, bool pdl, cudaStream_t s, int* n_launched);
+cudaError_t launch_plan(const PlanArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// The tcgen05 grouped GEMMs (cudaErrorNotSupported where a format has none).
+cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s);
+
+// Largest T for which the route kernels run the fused single-CTA select+plan.
+constexpr int kSmallT = 32;
+
+}  // namespace moe

@@ -1,0 +1,479 @@
+// C-ABI host layer: argument validation, workspace layout, launch sequencing.
+// Every stage is enqueued on the caller's stream with programmatic dependent
+// launch, so a kernel's launch overlaps the tail of the one before it; each
+// kernel waits (griddepcontrol.wait) before it reads anything.
+#include <cstdarg>
+#include <cstdio>
+#include <map>
+#include <mutex>
+#include <string>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace moe {
+
+__device__ int g_err_word;   // the library's device error word (one per device)
+
+const DeviceInfo& device_info() {
+    static std::mutex mu;
+    static std::map<int, DeviceInfo> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+    DeviceInfo di{};
+    cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.err_word), g_err_word) != cudaSuccess)
+        di.err_word = nullptr;
+    if (di.sm_count <= 0) di.sm_count = 1;
+    return cache.emplace(dev, di).first->second;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local int g_launches = 0;      // kernels launched by the thread's last successful call
+struct Hook {
+    cudaEvent_t begin = nullptr, end = nullptr;
+    int stage = -1;
+};
+thread_local Hook g_hook;
+std::mutex g_dispatch_mu;
+int g_dispatch = MOE_DISPATCH_AUTO;
+
+// Token counts up to this use the weight-streaming GEMV under MOE_DISPATCH_AUTO.
+constexpr int kGemvMaxT = 64;
+
+moe_status fail(moe_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+moe_status check_dims(const moe_dims* d) {
+    if (!d) return fail(MOE_ERR_NULL, "dims is NULL");
+    if (d->T < 0) return fail(MOE_ERR_SHAPE, "T = %d < 0", d->T);
+    if (d->H < 64 || d->H > 16384 || d->H % 64)
+        return fail(MOE_ERR_SHAPE, "H = %d: need 64 <= H <= 16384 and H %% 64 == 0", d->H);
+    if (d->I < 64 || d->I > 16384 || d->I % 64)
+        return fail(MOE_ERR_SHAPE, "I = %d: need 64 <= I <= 16384 and I %% 64 == 0", d->I);
+    if (d->E < 1 || d->E > 256) return fail(MOE_ERR_SHAPE, "E = %d: need 1 <= E <= 256", d->E);
+    if (d->k < 1 || d->k > d->E || d->k > 32)
+        return fail(MOE_ERR_SHAPE, "k = %d: need 1 <= k <= min(E, 32)", d->k);
+    if ((long long)d->T * d->k >= (1ll << 31)) return fail(MOE_ERR_SHAPE, "T * k >= 2^31");
+    return MOE_OK;
+}
+
+moe_status check_fmt(int32_t fmt) {
+    if (fmt != MOE_W_BF16 && fmt != MOE_W_AFFINE4_G64)
+        return fail(MOE_ERR_UNSUPPORTED, "weight format %d", fmt);
+    return MOE_OK;
+}
+
+void layout(const moe_dims* d, moe_ws_layout* L) {
+    const size_t T = d->T, H = d->H, E = d->E, P = (size_t)d->T * d->k, I = d->I;
+    size_t off = 0;
+    L->y_acc = off;
+    off = align256(off + T * H * 4);
+    L->h = off;
+    off = align256(off + P * I * 2);
+    L->xs = off;
+    off = align256(off + P * H * 2);
+    L->scratch = off;
+    off = align256(off + (size_t)kSmallT * E * 4 + 4096);
+    L->total = off;
+}
+
+struct WsView {
+    float* y_acc;
+    uint16_t* h;
+    uint16_t* xs;
+    float* l_scratch;
+};
+
+moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
+    moe_ws_layout L;
+    layout(d, &L);
+    if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_ALIGN, "workspace not 256-byte aligned");
+    if (ws_bytes < L.total)
+        return fail(MOE_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+    char* b = static_cast<char*>(ws);
+    v->y_acc = reinterpret_cast<float*>(b + L.y_acc);
+    v->h = reinterpret_cast<uint16_t*>(b + L.h);
+    v->xs = reinterpret_cast<uint16_t*>(b + L.xs);
+    v->l_scratch = reinterpret_cast<float*>(b + L.scratch);
+    return MOE_OK;
+}
+
+moe_status check_plan(const moe_plan_t* plan) {
+    if (!plan) return fail(MOE_ERR_NULL, "plan is NULL");
+    if (!plan->counts || !plan->offsets || !plan->perm || !plan->inv || !plan->tiles)
+        return fail(MOE_ERR_NULL, "a plan array is NULL");
+    return MOE_OK;
+}
+
+moe_status check_weights(const moe_experts_w* W) {
+    if (!W) return fail(MOE_ERR_NULL, "weights struct is NULL");
+    if (W->act != MOE_ACT_SWIGLU && W->act != MOE_ACT_RELU2)
+        return fail(MOE_ERR_UNSUPPORTED, "activation %d", W->act);
+    moe_status st = check_fmt(W->fmt);
+    if (st != MOE_OK) return st;
+    if (!W->w1 || !W->w2) return fail(MOE_ERR_NULL, "w1 or w2 is NULL");
+    if (!aligned16(W->w1) || !aligned16(W->w2)) return fail(MOE_ERR_ALIGN, "w1/w2 not 16-byte aligned");
+    if (W->fmt == MOE_W_AFFINE4_G64) {
+        if (!W->w1_scale || !W->w1_bias || !W->w2_scale || !W->w2_bias)
+            return fail(MOE_ERR_NULL, "affine-4 scale/bias pointer is NULL");
+        if (!aligned16(W->w1_scale) || !aligned16(W->w1_bias) || !aligned16(W->w2_scale) ||
+            !aligned16(W->w2_bias))
+            return fail(MOE_ERR_ALIGN, "affine-4 scale/bias not 16-byte aligned");
+    }
+    return MOE_OK;
+}
+
+moe_status check_route_args(const void* x, const float* logits, const float* w_router,
+                            const moe_dims* d, int32_t* idx, float* w) {
+    if ((x == nullptr) == (logits == nullptr))
+        return fail(MOE_ERR_NULL, "give exactly one of x or logits");
+    if (x && !w_router) return fail(MOE_ERR_NULL, "w_router is NULL (routing from x)");
+    if (!idx || !w) return fail(MOE_ERR_NULL, "topk_idx or topk_w is NULL");
+    if (x && (!aligned16(x) || !aligned16(w_router)))
+        return fail(MOE_ERR_ALIGN, "x / w_router not 16-byte aligned");
+    (void)d;
+    return MOE_OK;
+}
+
+int current_dispatch() {
+    std::lock_guard<std::mutex> lock(g_dispatch_mu);
+    return g_dispatch;
+}
+
+bool use_gemv(const moe_dims* d) {
+    const int mode = current_dispatch();
+    if (mode == MOE_DISPATCH_GEMV) return true;
+    if (mode == MOE_DISPATCH_GEMM) return false;
+    return d->T <= kGemvMaxT;
+}
+
+ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* topk_w,
+                            const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
+                            const WsView& v) {
+    ExpertArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.topk_w = topk_w;
+    a.counts = plan->counts;
+    a.offsets = plan->offsets;
+    a.perm = plan->perm;
+    a.tiles = plan->tiles;
+    a.T = d->T;
+    a.H = d->H;
+    a.E = d->E;
+    a.k = d->k;
+    a.I = d->I;
+    a.act = W->act;
+    a.fmt = W->fmt;
+    a.w1 = W->w1;
+    a.w1_scale = static_cast<const uint16_t*>(W->w1_scale);
+    a.w1_bias = static_cast<const uint16_t*>(W->w1_bias);
+    a.w2 = W->w2;
+    a.w2_scale = static_cast<const uint16_t*>(W->w2_scale);
+    a.w2_bias = static_cast<const uint16_t*>(W->w2_bias);
+    a.h = v.h;
+    a.xs = v.xs;
+    a.y_acc = v.y_acc;
+    a.y = static_cast<uint16_t*>(y);
+    a.out_scale = out_scale;
+    a.err = device_info().err_word;
+    return a;
+}
+
+// Event record that also works under stream capture (an event node there).
+cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return e;
+    if (cs == cudaStreamCaptureStatusActive) return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+    return cudaEventRecord(ev, s);
+}
+
+// Enqueues stages on one stream; records the one-shot hook's events around
+// the hooked stage and counts kernels.
+struct Seq {
+    cudaStream_t s;
+    int n = 0;
+    template <class F>
+    cudaError_t stage(int id, F&& f) {   // f(int* launched) -> cudaError_t
+        const bool hooked = g_hook.stage == id && g_hook.begin && g_hook.end;
+        cudaError_t e;
+        if (hooked && (e = record_event(g_hook.begin, s)) != cudaSuccess) return e;
+        int launched = 1;
+        if ((e = f(&launched)) != cudaSuccess) return e;
+        n += launched;
+        if (hooked) {
+            e = record_event(g_hook.end, s);
+            g_hook = Hook{};
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+};
+
+moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
+    const bool gemv = use_gemv(d);
+    cudaError_t e = q.stage(MOE_STAGE_UP, [&](int*) {
+        return gemv ? launch_gemv_up(a, true, q.s) : launch_gemm_up(a, true, q.s);
+    });
+    if (e == cudaErrorNotSupported)
+        return fail(MOE_ERR_UNSUPPORTED, "no expert kernel for this format/path in this build");
+    if (e != cudaSuccess) return cuda_fail(e, "expert up kernel");
+    e = q.stage(MOE_STAGE_DOWN, [&](int*) {
+        return gemv ? launch_gemv_down(a, true, q.s) : launch_gemm_down(a, true, q.s);
+    });
+    if (e == cudaErrorNotSupported)
+        return fail(MOE_ERR_UNSUPPORTED, "no expert kernel for this format/path in this build");
+    if (e != cudaSuccess) return cuda_fail(e, "expert down kernel");
+    e = q.stage(MOE_STAGE_FINAL, [&](int*) { return launch_finalize(a, true, q.s); });
+    if (e != cudaSuccess) return cuda_fail(e, "finalize");
+    return MOE_OK;
+}
+
+PlanArgs make_plan_args(const int32_t* idx, const moe_dims* d, const moe_plan_t* plan) {
+    PlanArgs p{};
+    p.idx = idx;
+    p.P = d->T * d->k;
+    p.E = d->E;
+    p.k = d->k;
+    p.counts = plan->counts;
+    p.offsets = plan->offsets;
+    p.perm = plan->perm;
+    p.inv = plan->inv;
+    p.tiles = plan->tiles;
+    p.err = device_info().err_word;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt) {
+    if (check_dims(d) != MOE_OK || check_fmt(fmt) != MOE_OK) return 0;
+    moe_ws_layout L;
+    layout(d, &L);
+    return L.total;
+}
+
+moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* out) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if ((st = check_fmt(fmt)) != MOE_OK) return st;
+    if (!out) return fail(MOE_ERR_NULL, "out is NULL");
+    layout(d, out);
+    return MOE_OK;
+}
+
+moe_status moe_route(const void* x, const float* logits, const float* w_router,
+                     const float* expert_bias, const moe_dims* d, float eps, float scale,
+                     int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
+    if ((st = check_route_args(x, logits, w_router, d, topk_idx, topk_w)) != MOE_OK) return st;
+    RouteArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.logits = logits;
+    a.w_router = w_router;
+    a.bias = expert_bias;
+    a.T = d->T;
+    a.H = d->H;
+    a.E = d->E;
+    a.k = d->k;
+    a.eps = eps;
+    a.scale = scale;
+    a.idx = topk_idx;
+    a.w = topk_w;
+    a.err = device_info().err_word;
+    Seq q{reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = q.stage(MOE_STAGE_ROUTE, [&](int* n) { return launch_route(a, false, true, q.s, n); });
+    if (e != cudaSuccess) return cuda_fail(e, "route");
+    g_launches = q.n;
+    return MOE_OK;
+}
+
+moe_status moe_plan(const int32_t* topk_idx, const moe_dims* d, const moe_plan_t* plan, void* ws,
+                    size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
+    if (!topk_idx) return fail(MOE_ERR_NULL, "topk_idx is NULL");
+    if ((st = check_plan(plan)) != MOE_OK) return st;
+    WsView v;
+    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    const PlanArgs p = make_plan_args(topk_idx, d, plan);
+    Seq q{reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = q.stage(MOE_STAGE_PLAN, [&](int*) { return launch_plan(p, true, q.s); });
+    if (e != cudaSuccess) return cuda_fail(e, "plan");
+    g_launches = q.n;
+    return MOE_OK;
+}
+
+moe_status moe_experts(const void* x, const moe_plan_t* plan, const float* topk_w,
+                       const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
+                       void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
+    if (!x || !topk_w || !y) return fail(MOE_ERR_NULL, "x, topk_w or y is NULL");
+    if (!aligned16(x) || !aligned16(y)) return fail(MOE_ERR_ALIGN, "x or y not 16-byte aligned");
+    if ((st = check_plan(plan)) != MOE_OK) return st;
+    if ((st = check_weights(W)) != MOE_OK) return st;
+    WsView v;
+    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    Seq q{reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = launch_zero(v.y_acc, (size_t)d->T * d->H, true, q.s);
+    if (e != cudaSuccess) return cuda_fail(e, "zero y_acc");
+    q.n = 1;
+    const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    if ((st = run_experts(q, a, d)) != MOE_OK) return st;
+    g_launches = q.n;
+    return MOE_OK;
+}
+
+moe_status moe_forward(const void* x, const float* logits, const float* w_router,
+                       const float* expert_bias, const moe_dims* d, float eps, float router_scale,
+                       float out_scale, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
+                       const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
+    if (!x || !y) return fail(MOE_ERR_NULL, "x or y is NULL (both are needed by the experts)");
+    if (!aligned16(x) || !aligned16(y)) return fail(MOE_ERR_ALIGN, "x or y not 16-byte aligned");
+    if (!logits && !w_router) return fail(MOE_ERR_NULL, "w_router is NULL (routing from x)");
+    if (!topk_idx || !topk_w) return fail(MOE_ERR_NULL, "topk_idx or topk_w is NULL");
+    if (!logits && !aligned16(w_router)) return fail(MOE_ERR_ALIGN, "w_router not 16-byte aligned");
+    if ((st = check_plan(plan)) != MOE_OK) return st;
+    if ((st = check_weights(W)) != MOE_OK) return st;
+    WsView v;
+    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+
+    RouteArgs r{};
+    r.x = logits ? nullptr : static_cast<const uint16_t*>(x);
+    r.logits = logits;
+    r.w_router = w_router;
+    r.bias = expert_bias;
+    r.l_scratch = v.l_scratch;
+    r.T = d->T;
+    r.H = d->H;
+    r.E = d->E;
+    r.k = d->k;
+    r.eps = eps;
+    r.scale = router_scale;
+    r.idx = topk_idx;
+    r.w = topk_w;
+    r.counts = plan->counts;
+    r.offsets = plan->offsets;
+    r.perm = plan->perm;
+    r.inv = plan->inv;
+    r.tiles = plan->tiles;
+    r.zero_ptr = v.y_acc;              // the router also clears the fp32 accumulator
+    r.zero_count = (size_t)d->T * d->H;
+    r.err = device_info().err_word;
+    const bool fuse = d->T <= kSmallT;  // one CTA routes and plans all pairs
+    Seq q{reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = q.stage(MOE_STAGE_ROUTE, [&](int* n) { return launch_route(r, fuse, true, q.s, n); });
+    if (e != cudaSuccess) return cuda_fail(e, "route");
+    if (!fuse) {
+        const PlanArgs p = make_plan_args(topk_idx, d, plan);
+        e = q.stage(MOE_STAGE_PLAN, [&](int*) { return launch_plan(p, true, q.s); });
+        if (e != cudaSuccess) return cuda_fail(e, "plan");
+    }
+    const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    if ((st = run_experts(q, a, d)) != MOE_OK) return st;
+    g_launches = q.n;
+    return MOE_OK;
+}
+
+moe_status moe_forward_host(const void* x_host, void* x_dev, const float* w_router,
+                            const float* expert_bias, const moe_dims* d, float eps,
+                            float router_scale, float out_scale, const moe_experts_w* W,
+                            int32_t* topk_idx, float* topk_w, const moe_plan_t* plan, void* y_dev,
+                            void* y_host, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->T == 0) return MOE_OK;   // empty batch: nothing to do
+    if (!x_host || !y_host || !x_dev) return fail(MOE_ERR_NULL, "x_host, x_dev or y_host is NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t bytes = (size_t)d->T * d->H * 2;
+    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
+    st = moe_forward(x_dev, nullptr, w_router, expert_bias, d, eps, router_scale, out_scale, W,
+                     topk_idx, topk_w, plan, y_dev, ws, ws_bytes, stream);
+    if (st != MOE_OK) return st;
+    e = cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy y to host");
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    return MOE_OK;
+}
+
+int32_t moe_set_dispatch(int32_t mode) {
+    std::lock_guard<std::mutex> lock(g_dispatch_mu);
+    const int old = g_dispatch;
+    if (mode == MOE_DISPATCH_AUTO || mode == MOE_DISPATCH_GEMV || mode == MOE_DISPATCH_GEMM)
+        g_dispatch = mode;
+    return old;
+}
+
+moe_status moe_device_error(int32_t* code, moe_stream_t stream) {
+    if (!code) return fail(MOE_ERR_NULL, "code is NULL");
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, moe::g_err_word, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(moe::g_err_word, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    *code = v;
+    if (v != 0) return fail(MOE_ERR_DEVICE, "device error code %d", v);
+    return MOE_OK;
+}
+
+moe_status moe_profile_hook(void* ev_begin, void* ev_end, int32_t stage) {
+    if (!ev_begin || !ev_end) {
+        g_hook = Hook{};
+        return MOE_OK;
+    }
+    if (stage < MOE_STAGE_ROUTE || stage > MOE_STAGE_FINAL) return fail(MOE_ERR_UNSUPPORTED, "stage %d", stage);
+    g_hook.begin = static_cast<cudaEvent_t>(ev_begin);
+    g_hook.end = static_cast<cudaEvent_t>(ev_end);
+    g_hook.stage = stage;
+    return MOE_OK;
+}
+
+int32_t moe_last_launch_count(void) { return g_launches; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

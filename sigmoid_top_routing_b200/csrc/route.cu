@@ -1,0 +1,368 @@
+// Sigmoid router with a selection-only expert bias and normalised top-k.
+//
+// TileGym PR #187 ("[E2E Model Support] Add TileGym kernel integration for
+// LFM2 MoE"), section "Weight layout and routing": sigmoid scores, the bias
+// only chooses the experts, the gathered weights stay unbiased, norm_topk
+// divides by sum + 1e-6 and then routed_scaling_factor multiplies.
+// TensorFold pull #1492, "What": fp32 router weights; "Verification": an
+// all-NaN router row must never pick the same expert twice.
+//
+// Logits are fp32 FMA chains in one fixed order, the same in every kernel
+// here, so a token's logits (and so its picks and weights) do not depend on
+// how many tokens share the launch:
+//   H is cut into chunks of 32 consecutive h; segment w (0..7) holds chunks
+//   c with c % 8 == w; p_w is an fmaf chain over segment w in increasing h,
+//   starting at 0; L = p_0 + p_1 + ... + p_7, left to right.
+//
+// Selection: a warp per token; each lane holds experts lane, lane+32, ...;
+// k rounds of a warp-wide max over 64-bit keys (score key, ~expert id).  The
+// score key orders c = s + bias with NaN below every number and -0 == +0;
+// a picked expert's key drops below every NaN key, so picks stay distinct
+// even when every score is NaN (the row then picks 0, 1, ..., k-1).
+#include "common.cuh"
+#include "internal.h"
+#include "launch.h"
+#include "plan_dev.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kSegs = 8;      // segments of the canonical logit order (= warps per CTA)
+constexpr int kChunk = 32;    // h per chunk
+
+MOE_DEV uint32_t score_key(float c) {
+    if (c != c) return 0u;                      // NaN: below every number
+    if (c == 0.0f) c = 0.0f;                    // -0 -> +0
+    uint32_t u = __float_as_uint(c);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+MOE_DEV float sigmoid_f32(float L) { return 1.0f / (1.0f + expf(-L)); }
+
+// Picks and weights of one token.  Lv[i] is the logit of expert lane + 32 i.
+// Lane j (< k) returns slot j's expert in *e_out (and writes idx/w rows).
+template <int NE>
+MOE_DEV int select_token(const float (&Lv)[NE], const float* __restrict__ bias, int E, int k,
+                         float eps, float scale, int32_t* idx_row, float* w_row) {
+    const int lane = threadIdx.x & 31;
+    float s[NE];
+    uint32_t khi[NE], klo[NE];
+#pragma unroll
+    for (int i = 0; i < NE; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+            s[i] = sigmoid_f32(Lv[i]);
+            const float c = s[i] + (bias ? __ldg(bias + e) : 0.0f);
+            khi[i] = score_key(c);
+            klo[i] = 0xFFFFFFFFu - (uint32_t)e;
+        } else {
+            s[i] = 0.0f;
+            khi[i] = 0u;
+            klo[i] = 0u;
+        }
+    }
+    int my_e = 0;
+    float my_s = 0.0f, sum = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bh = khi[0], bl = klo[0];
+#pragma unroll
+        for (int i = 1; i < NE; ++i)
+            if (khi[i] > bh || (khi[i] == bh && klo[i] > bl)) { bh = khi[i]; bl = klo[i]; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t oh = __shfl_xor_sync(0xffffffffu, bh, o);
+            const uint32_t ol = __shfl_xor_sync(0xffffffffu, bl, o);
+            if (oh > bh || (oh == bh && ol > bl)) { bh = oh; bl = ol; }
+        }
+        const int ej = (int)(0xFFFFFFFFu - bl);
+        const int owner = ej & 31, ii = ej >> 5;
+        float mine = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (i == ii) mine = s[i];
+        if (lane == owner) {
+#pragma unroll
+            for (int i = 0; i < NE; ++i)
+                if (i == ii) { khi[i] = 0u; klo[i] = 0u; }
+        }
+        const float sj = __shfl_sync(0xffffffffu, mine, owner);
+        if (lane == j) { my_e = ej; my_s = sj; }
+        sum += sj;                                 // slot order
+    }
+    const float denom = sum + eps;
+    if (lane < k) {
+        idx_row[lane] = my_e;
+        w_row[lane] = my_s / denom * scale;
+    }
+    return my_e;
+}
+
+MOE_DEV void zero_slice(const RouteArgs& a) {
+    if (!a.zero_ptr) return;
+    const size_t n4 = a.zero_count / 4;
+    float4* p = reinterpret_cast<float4*>(a.zero_ptr);
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
+        p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// Small T (<= 32): one CTA per expert.  Warp w computes segment w's chain for
+// every token (lane = token); the 8 partials are summed in order.
+__global__ void __launch_bounds__(256) k_logits_small(RouteArgs a) {
+    extern __shared__ float sm[];
+    float* wr = sm;                       // H floats: this expert's router row
+    float* part = sm + a.H;               // 8 x 32
+    pdl_wait();
+    zero_slice(a);
+    const int e = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float4* src = reinterpret_cast<const float4*>(a.w_router + (size_t)e * a.H);
+    for (int i = threadIdx.x; i < a.H / 4; i += blockDim.x) reinterpret_cast<float4*>(wr)[i] = __ldg(src + i);
+    __syncthreads();
+    float acc = 0.0f;
+    if (lane < a.T) {
+        const uint16_t* xr = a.x + (size_t)lane * a.H;
+        for (int c = warp; c < a.H / kChunk; c += kSegs) {
+#pragma unroll
+            for (int q = 0; q < kChunk / 8; ++q) {
+                const int h = c * kChunk + q * 8;
+                const uint4 xv = ld_nc(xr + h);
+                acc = fmaf(bf16lo(xv.x), wr[h + 0], acc);
+                acc = fmaf(bf16hi(xv.x), wr[h + 1], acc);
+                acc = fmaf(bf16lo(xv.y), wr[h + 2], acc);
+                acc = fmaf(bf16hi(xv.y), wr[h + 3], acc);
+                acc = fmaf(bf16lo(xv.z), wr[h + 4], acc);
+                acc = fmaf(bf16hi(xv.z), wr[h + 5], acc);
+                acc = fmaf(bf16lo(xv.w), wr[h + 6], acc);
+                acc = fmaf(bf16hi(xv.w), wr[h + 7], acc);
+            }
+        }
+    }
+    part[warp * 32 + lane] = acc;
+    __syncthreads();
+    if (warp == 0 && lane < a.T) {
+        float L = part[lane];
+#pragma unroll
+        for (int w = 1; w < kSegs; ++w) L += part[w * 32 + lane];
+        a.l_scratch[(size_t)lane * a.E + e] = L;
+    }
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// Selection from fp32 logits in memory; FUSE also builds the plan (one CTA,
+// T <= 32 so P <= 1024).
+template <int NE, bool FUSE>
+__global__ void __launch_bounds__(256) k_select(RouteArgs a) {
+    __shared__ int s_idx[FUSE ? 1024 : 1];
+    __shared__ int s_cnt[FUSE ? 256 : 1], s_off[FUSE ? 257 : 1], s_til[FUSE ? 257 : 1];
+    __shared__ int s_cur[FUSE ? 256 : 1], s_wcnt[FUSE ? 8 * 256 : 1];
+    pdl_wait();
+    zero_slice(a);
+    const float* L = a.logits ? a.logits : a.l_scratch;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int t = blockIdx.x * 8 + warp; t < a.T; t += gridDim.x * 8) {
+        float Lv[NE];
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            Lv[i] = e < a.E ? L[(size_t)t * a.E + e] : 0.0f;
+        }
+        const int e = select_token<NE>(Lv, a.bias, a.E, a.k, a.eps, a.scale, a.idx + (size_t)t * a.k,
+                                       a.w + (size_t)t * a.k);
+        if (FUSE && lane < a.k) s_idx[t * a.k + lane] = e;
+    }
+    if (FUSE) {
+        const int P = a.T * a.k, E = a.E;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) s_cnt[i] = 0;
+        for (int i = threadIdx.x; i < 8 * 256; i += blockDim.x) s_wcnt[i] = 0;
+        __syncthreads();
+        for (int p = threadIdx.x; p < P; p += blockDim.x) atomicAdd(&s_cnt[s_idx[p]], 1);
+        __syncthreads();
+        if (warp == 0) warp_exclusive_scan(s_cnt, s_off, E, 0);
+        if (warp == 1) warp_exclusive_scan(s_cnt, s_til, E, kTileM);
+        __syncthreads();
+        for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+            a.offsets[e] = s_off[e];
+            a.tiles[e] = s_til[e];
+            if (e < E) {
+                a.counts[e] = s_cnt[e];
+                s_cur[e] = s_off[e];
+            }
+        }
+        __syncthreads();
+        stable_scatter<8>(s_idx, P, E, s_cur, s_wcnt, a.perm, a.inv);
+    }
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// Large T: TT tokens per CTA.  Warp w computes segment w for all TT tokens
+// and all experts (lane holds experts lane + 32 i), staging the router chunk
+// (transposed) and the token chunk (fp32) in its own shared memory; then the
+// 8 partials are summed in order and each warp selects for TT / 8 tokens.
+template <int NE, int TT, int HCH>
+__global__ void __launch_bounds__(256) k_route_large(RouteArgs a) {
+    extern __shared__ float sm[];
+    constexpr int EP = 32 * NE;
+    constexpr int WARP_FLOATS = HCH * EP + HCH * TT;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float* wt = sm + warp * WARP_FLOATS;          // [HCH][EP]
+    float* xs = wt + HCH * EP;                    // [HCH][TT]
+    pdl_wait();
+    zero_slice(a);
+    const int t0 = blockIdx.x * TT;
+    const int E = a.E, H = a.H;
+
+    float acc[TT][NE];
+#pragma unroll
+    for (int m = 0; m < TT; ++m)
+#pragma unroll
+        for (int i = 0; i < NE; ++i) acc[m][i] = 0.0f;
+
+    for (int c = warp; c < H / kChunk; c += kSegs) {
+#pragma unroll
+        for (int half = 0; half < kChunk / HCH; ++half) {
+            const int h0 = c * kChunk + half * HCH;
+            // stage router chunk transposed: wt[hh][e]
+#pragma unroll
+            for (int i = 0; i < NE; ++i) {
+                const int e = lane + 32 * i;
+                if (e < E) {
+                    const float4* src = reinterpret_cast<const float4*>(a.w_router + (size_t)e * H + h0);
+#pragma unroll
+                    for (int q = 0; q < HCH / 4; ++q) {
+                        const float4 v = __ldg(src + q);
+                        wt[(4 * q + 0) * EP + e] = v.x;
+                        wt[(4 * q + 1) * EP + e] = v.y;
+                        wt[(4 * q + 2) * EP + e] = v.z;
+                        wt[(4 * q + 3) * EP + e] = v.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int hh = 0; hh < HCH; ++hh) wt[hh * EP + e] = 0.0f;
+                }
+            }
+            // stage token chunk: xs[hh][t]
+            if (lane < TT) {
+                const int t = t0 + lane;
+                if (t < a.T) {
+                    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * H + h0);
+#pragma unroll
+                    for (int q = 0; q < HCH / 8; ++q) {
+                        const uint4 v = ld_nc(src + q);
+                        xs[(8 * q + 0) * TT + lane] = bf16lo(v.x);
+                        xs[(8 * q + 1) * TT + lane] = bf16hi(v.x);
+                        xs[(8 * q + 2) * TT + lane] = bf16lo(v.y);
+                        xs[(8 * q + 3) * TT + lane] = bf16hi(v.y);
+                        xs[(8 * q + 4) * TT + lane] = bf16lo(v.z);
+                        xs[(8 * q + 5) * TT + lane] = bf16hi(v.z);
+                        xs[(8 * q + 6) * TT + lane] = bf16lo(v.w);
+                        xs[(8 * q + 7) * TT + lane] = bf16hi(v.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int hh = 0; hh < HCH; ++hh) xs[hh * TT + lane] = 0.0f;
+                }
+            }
+            __syncwarp();
+#pragma unroll 4
+            for (int hh = 0; hh < HCH; ++hh) {
+                float wv[NE];
+#pragma unroll
+                for (int i = 0; i < NE; ++i) wv[i] = wt[hh * EP + lane + 32 * i];
+                const float4* x4 = reinterpret_cast<const float4*>(xs + hh * TT);
+#pragma unroll
+                for (int m4 = 0; m4 < TT / 4; ++m4) {
+                    const float4 xv = x4[m4];
+#pragma unroll
+                    for (int i = 0; i < NE; ++i) {
+                        acc[4 * m4 + 0][i] = fmaf(xv.x, wv[i], acc[4 * m4 + 0][i]);
+                        acc[4 * m4 + 1][i] = fmaf(xv.y, wv[i], acc[4 * m4 + 1][i]);
+                        acc[4 * m4 + 2][i] = fmaf(xv.z, wv[i], acc[4 * m4 + 2][i]);
+                        acc[4 * m4 + 3][i] = fmaf(xv.w, wv[i], acc[4 * m4 + 3][i]);
+                    }
+                }
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    float* part = sm;                              // [8][TT][EP]
+#pragma unroll
+    for (int m = 0; m < TT; ++m)
+#pragma unroll
+        for (int i = 0; i < NE; ++i) part[(warp * TT + m) * EP + lane + 32 * i] = acc[m][i];
+    __syncthreads();
+    for (int m = warp; m < TT; m += kSegs) {
+        const int t = t0 + m;
+        if (t >= a.T) break;
+        float Lv[NE];
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            float L = part[(0 * TT + m) * EP + e];
+#pragma unroll
+            for (int w = 1; w < kSegs; ++w) L += part[(w * TT + m) * EP + e];
+            Lv[i] = L;
+        }
+        select_token<NE>(Lv, a.bias, E, a.k, a.eps, a.scale, a.idx + (size_t)t * a.k,
+                         a.w + (size_t)t * a.k);
+    }
+    pdl_trigger();
+}
+
+template <int NE, int TT, int HCH>
+cudaError_t run_large(const RouteArgs& a, bool pdl, cudaStream_t s) {
+    constexpr int EP = 32 * NE;
+    size_t stage = (size_t)8 * (HCH * EP + HCH * TT) * sizeof(float);
+    size_t part = (size_t)8 * TT * EP * sizeof(float);
+    size_t smem = stage > part ? stage : part;
+    auto kern = k_route_large<NE, TT, HCH>;
+    cudaError_t e = ensure_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3((a.T + TT - 1) / TT), dim3(256), smem, s, pdl, a);
+}
+
+template <int NE>
+cudaError_t run_select(const RouteArgs& a, bool fuse, bool pdl, cudaStream_t s) {
+    if (fuse) return launch_k(k_select<NE, true>, dim3(1), dim3(256), 0, s, pdl, a);
+    return launch_k(k_select<NE, false>, dim3((a.T + 7) / 8), dim3(256), 0, s, pdl, a);
+}
+
+cudaError_t dispatch_select(const RouteArgs& a, bool fuse, bool pdl, cudaStream_t s) {
+    if (a.E <= 32) return run_select<1>(a, fuse, pdl, s);
+    if (a.E <= 64) return run_select<2>(a, fuse, pdl, s);
+    if (a.E <= 128) return run_select<4>(a, fuse, pdl, s);
+    return run_select<8>(a, fuse, pdl, s);
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteArgs& a, bool fuse_plan, bool pdl, cudaStream_t s, int* n_launched) {
+    *n_launched = 0;
+    if (a.T == 0) return cudaSuccess;
+    *n_launched = 1;
+    const bool small = a.T <= kSmallT;
+    if (a.logits) return dispatch_select(a, fuse_plan && small, pdl, s);
+    if (small && a.l_scratch) {
+        // two launches: per-expert logits into scratch (this one also zeroes
+        // the accumulator), then select (+ plan)
+        size_t smem = (size_t)a.H * sizeof(float) + 8 * 32 * sizeof(float);
+        cudaError_t e = ensure_smem(k_logits_small, smem);
+        if (e != cudaSuccess) return e;
+        e = launch_k(k_logits_small, dim3(a.E), dim3(256), smem, s, pdl, a);
+        if (e != cudaSuccess) return e;
+        *n_launched = 2;
+        RouteArgs b = a;
+        b.zero_ptr = nullptr;
+        return dispatch_select(b, fuse_plan, pdl, s);
+    }
+    if (a.E <= 32) return run_large<1, 32, 32>(a, pdl, s);
+    if (a.E <= 64) return run_large<2, 32, 32>(a, pdl, s);
+    if (a.E <= 128) return run_large<4, 16, 32>(a, pdl, s);
+    return run_large<8, 8, 16>(a, pdl, s);
+}
+
+}  // namespace moe
