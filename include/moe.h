@@ -204,6 +204,34 @@ MOE_API moe_status moe_profile_hook(void* ev_begin, void* ev_end, int32_t stage)
 /* Number of kernels the calling thread's last successful moe_* call launched. */
 MOE_API int32_t moe_last_launch_count(void);
 
+/* moe_forward for callers that cannot allocate device memory.  (The pages
+ * have no counterpart: this is an interface choice of this library.)
+ * Some callers have no workspace to give: a plugin host that hands a custom
+ * op only its input and output tensors, code running inside another
+ * framework's CUDA-graph capture (where cudaMalloc cannot be captured and may
+ * synchronise the device), or a latency-bound serving loop that must never
+ * wait on an allocator.  This call takes the same arguments as moe_forward
+ * minus ws/ws_bytes: its scratch (fp32 accumulator, bf16 activations, router
+ * logits) is one fixed 16 MiB device array inside the library, which every GPU
+ * that loads the library holds until the process exits.  It allocates
+ * nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - Sizes whose scratch exceeds 16 MiB (T*H*4 + T*k*I*2 + 32*E*4 + 4 KiB,
+ *     each rounded up to 256 bytes) are refused with MOE_ERR_WORKSPACE and a
+ *     message giving the bytes needed.  Runs bf16 weights only, always on the
+ *     weight-streaming grouped GEMV (MOE_ERR_UNSUPPORTED for affine 4-bit).
+ *   - The first call on a device looks up the array's device address on that
+ *     device (cudaGetSymbolAddress, once per device, with the device current);
+ *     make that first call before any stream capture.
+ *   - Every call shares the array and it keeps the last call's contents (the
+ *     accumulator is cleared at the start of each call).  Calls whose work
+ *     overlaps on the GPU (other streams, other threads) race on it: run them
+ *     one after another on one stream. */
+MOE_API moe_status moe_forward_static(const void* x, const float* logits, const float* w_router,
+                                      const float* expert_bias, const moe_dims* d, float eps,
+                                      float router_scale, float out_scale, const moe_experts_w* W,
+                                      int32_t* topk_idx, float* topk_w, const moe_plan_t* plan,
+                                      void* y, moe_stream_t stream);
+
 /* Process-wide choice of expert kernels (moe_dispatch); returns the old one. */
 MOE_API int32_t moe_set_dispatch(int32_t mode);
 

@@ -59,6 +59,9 @@ PROTOTYPES = {
     "moe_forward_host": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float,
                                    c_float, c_float, POINTER(moe_experts_w), c_void_p, c_void_p,
                                    POINTER(moe_plan_t), c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_forward_static": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float,
+                                     c_float, c_float, POINTER(moe_experts_w), c_void_p, c_void_p,
+                                     POINTER(moe_plan_t), c_void_p, c_void_p]),
     "moe_profile_hook": (c_int32, [c_void_p, c_void_p, c_int32]),
     "moe_last_launch_count": (c_int32, []),
     "moe_set_dispatch": (c_int32, [c_int32]),

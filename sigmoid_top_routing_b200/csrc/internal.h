@@ -80,4 +80,8 @@ cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s);
 // Largest T for which the route kernels run the fused single-CTA select+plan.
 constexpr int kSmallT = 32;
 
+// Thread-local status text and launch count of the C-ABI layer (moe_api.cu).
+void set_last_error(const char* msg);
+void set_last_launch_count(int n);
+
 }  // namespace moe

@@ -272,6 +272,12 @@ PlanArgs make_plan_args(const int32_t* idx, const moe_dims* d, const moe_plan_t*
 
 }  // namespace
 
+namespace moe {
+// For entry points defined in other files of the library.
+void set_last_error(const char* msg) { g_last_error = msg; }
+void set_last_launch_count(int n) { g_launches = n; }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt) {
