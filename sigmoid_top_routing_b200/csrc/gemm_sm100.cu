@@ -1,9 +1,507 @@
-// Prefill-sized grouped expert GEMMs on tcgen05 (filled in by the next step).
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// Swap-AB form: the expert's weight rows are the MMA's M = 128 operand (A,
+// streamed by TMA) and the expert's tokens are its N operand (B, N = 16..BN
+// in steps of 16), so an expert with 3 tokens costs an N = 16 MMA while its
+// weights stream at full rate, and an expert with 500 tokens runs 128 x 256
+// tiles.  D[feature][token] accumulates in fp32 in TMEM (double-buffered so
+// the epilogue overlaps the next tile's main loop).
+//
+//   up (SwiGLU):  a tile = 64 gate rows + 64 up rows of W1[e] (gate-first
+//                 layout, TileGym PR #187 "Weight layout and routing"); TMEM
+//                 lanes j and 64 + j hold gate and up of feature j, and the
+//                 epilogue writes h[pos, f] = bf16_rn(silu(g) * u).
+//   up (relu^2):  a tile = 128 rows of W1[e]; h = bf16_rn(relu(u)^2), NaN
+//                 kept (vllm.cpp PR #684; bloomery PR #235 "What").
+//   down:         a tile = 128 rows of W2[e]; y_acc[t, f] += w[p] * D (fp32
+//                 reductions), the weighted combine of the pages' MoeCombine.
+//
+// Prior art: the staged prompt kernels of TensorFold issue #548 ("Prompt rows
+// of the grouped experts: two forms": items of 64 pairs x 128 columns staged
+// through shared memory) -- kept: staged tiles and a pair's bits depending
+// only on its row and expert; changed for sm_100a: TMA, tcgen05, TMEM.
+//
+// Warp roles (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      producer: TMA for weights; token rows gathered with cp.async
+//               (up) or TMA (down, h is contiguous in plan order)
+//   warp 1      TMEM owner and MMA issuer (one thread)
+//   warps 2..5  epilogue (TMEM lanes 32 * (warp % 4) ...)
+// Every mbarrier wait is bounded; on expiry the kernel records error code 2,
+// drains what it issued, frees TMEM and returns.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
 #include "internal.h"
+#include "launch.h"
+#include "plan_dev.cuh"
+#include "sm100.cuh"
 
 namespace moe {
+namespace {
 
-cudaError_t launch_gemm_up(const ExpertArgs&, bool, cudaStream_t) { return cudaErrorNotSupported; }
-cudaError_t launch_gemm_down(const ExpertArgs&, bool, cudaStream_t) { return cudaErrorNotSupported; }
+using namespace sm100;
+
+constexpr int kBK = 64;                  // k per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kAStage = 128 * kBK * 2;   // 16 KB of weight rows per stage
+constexpr int kThreads = 192;
+
+enum Mode { kUpSwiglu = 0, kUpRelu2 = 1, kDown = 2 };
+
+struct GemmParams {
+    const int32_t* counts;
+    const int32_t* offsets;
+    const int32_t* perm;
+    const float* topk_w;
+    const uint16_t* x;       // (T, H) token rows (up)
+    uint16_t* h;             // (P, I) activations in plan order (written by up, read by down)
+    float* y_acc;            // (T, H) (down)
+    int E, k, H, I;
+    int K;                   // reduction length: H (up) or I (down)
+    int rows_per_expert;     // rows of the A tensor per expert: 2I, I or H
+    int feats;               // output features per expert: I (up) or H (down)
+    int* err;
+};
+
+template <int BN, int STAGES>
+struct Smem {
+    static constexpr int kBStage = BN * 128;
+    static constexpr size_t kA = 0;
+    static constexpr size_t kB = kA + size_t(STAGES) * kAStage;
+    static constexpr size_t kBar = kB + size_t(STAGES) * kBStage;           // 8-byte barriers
+    static constexpr int kNumBar = 2 * STAGES + 4 + 1;                      // full, empty, tfull[2], tempty[2], drain
+    static constexpr size_t kMisc = kBar + kNumBar * 8;                       // tmem base, abort flag
+    static constexpr size_t kTileBase = kMisc + 16;                           // 257 ints
+    static constexpr size_t kTok = kTileBase + 257 * 4;                       // BN ints (token of column)
+    static constexpr size_t kTokW = kTok + BN * 4;                            // BN floats
+    static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats
+    static constexpr size_t kEnd = kU + 64 * 17 * 4;
+    static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
+};
+
+struct Tile {
+    int e, wt, tt, ntok, n, row0;
+};
+
+// Tile t -> (expert, weight tile, token tile).  Tiles of one expert run
+// weight-tile-major with the token tiles innermost, so the CTAs working at
+// one time share weight tiles in L2.
+template <int BN>
+MOE_DEV Tile decode_tile(int t, const int* base, int E, const int32_t* counts, const int32_t* offsets) {
+    int lo = 0, hi = E;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (base[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    Tile r;
+    r.e = lo;
+    const int c = counts[lo];
+    const int ntt = (c + BN - 1) / BN;
+    const int local = t - base[lo];
+    r.wt = local / ntt;
+    r.tt = local % ntt;
+    r.ntok = min(BN, c - r.tt * BN);
+    r.n = (r.ntok + 15) & ~15;
+    r.row0 = offsets[lo] + r.tt * BN;
+    return r;
+}
+
+MOE_DEV void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+MOE_DEV void cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int MODE, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams g) {
+    using L = Smem<BN, STAGES>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* sA = sm + L::kA;
+    unsigned char* sB = sm + L::kB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::kMisc);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
+    int* s_base = reinterpret_cast<int*>(sm + L::kTileBase);
+    int* s_tok = reinterpret_cast<int*>(sm + L::kTok);
+    float* s_tokw = reinterpret_cast<float*>(sm + L::kTokW);
+    float* s_u = reinterpret_cast<float*>(sm + L::kU);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+    // up: 32 producer lanes gather token rows with cp.async, + 1 expect_tx arrive
+    constexpr uint32_t kFullCount = MODE == kDown ? 1 : 33;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], kFullCount);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(drain, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        if (MODE == kDown) tma_prefetch_desc(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    pdl_wait();   // the plan and (for down) h come from earlier kernels
+    // tile table: tiles of expert e = weight tiles x ceil(count / BN)
+    const int fpt = MODE == kUpSwiglu ? 64 : 128;      // output features per tile
+    const int n_wt = (g.feats + fpt - 1) / fpt;
+    if (warp == 2) {
+        const int per = (g.E + 31) / 32;
+        int local = 0;
+        for (int j = 0; j < per; ++j) {
+            const int e = lane * per + j;
+            if (e < g.E) local += n_wt * ((g.counts[e] + BN - 1) / BN);
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int j = 0; j < per; ++j) {
+            const int e = lane * per + j;
+            if (e < g.E) {
+                s_base[e] = run;
+                run += n_wt * ((g.counts[e] + BN - 1) / BN);
+            }
+        }
+        if (lane == 31) s_base[g.E] = incl;
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int total = s_base[g.E];
+    const int nkb = g.K / kBK;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t issued_mask = 0;            // stages with a fill whose arrival is not yet known
+        uint32_t issued_par = 0;             // parity of that fill
+        bool ok = true;
+        const uint64_t pol_w = policy_evict_first();
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            // token rows of this tile (up: gathered from x by pair)
+            const uint16_t* trow[BN / 32 > 0 ? BN / 32 : 1];
+            if (MODE != kDown) {
+#pragma unroll
+                for (int j = 0; j < (BN + 31) / 32; ++j) {
+                    const int r = lane + 32 * j;
+                    const int rr = r < tl.ntok ? r : (tl.ntok - 1);   // pad with a valid row
+                    const int p = g.perm[tl.row0 + rr];
+                    trow[j] = g.x + (size_t)(p / g.k) * g.H;
+                }
+            }
+            const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
+            for (int kb = 0; kb < nkb; ++kb) {
+                if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t bytes = kAStage + (MODE == kDown ? tl.n * 128 : 0);
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    unsigned char* a = sA + size_t(s) * kAStage;
+                    if (MODE == kUpSwiglu) {
+                        tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
+                        tma_load_2d_hint(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s], pol_w);
+                    } else {
+                        tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
+                    }
+                    if (MODE == kDown) {
+                        unsigned char* b = sB + size_t(s) * L::kBStage;
+                        for (int j = 0; j < tl.n / 16; ++j)
+                            tma_load_2d(b + j * 2048, &tmB, kb * kBK, tl.row0 + 16 * j, &full[s]);
+                    }
+                }
+                if (MODE != kDown) {
+                    // gather: row r, 16-byte chunk c -> swizzled (r, c ^ (r & 7))
+                    const uint32_t b = smem_u32(sB + size_t(s) * L::kBStage);
+#pragma unroll
+                    for (int j = 0; j < (BN + 31) / 32; ++j) {
+                        const int r = lane + 32 * j;
+                        if (r < tl.n) {
+                            const unsigned char* src = reinterpret_cast<const unsigned char*>(trow[j]) + kb * 128;
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                cp_async16(b + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16);
+                        }
+                    }
+                    cp_async_arrive(&full[s]);
+                }
+                issued_mask |= 1u << s;
+                issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+            }
+        }
+        if (!ok) {
+            if (lane == 0) report_error(g.err, kErrWaitExpired);
+            *s_abort = 1;
+        }
+        // wait (bounded) for every fill this warp issued to land before the CTA can exit
+        for (int q = 0; q < STAGES; ++q)
+            if (issued_mask >> q & 1u) mbar_wait(&full[q], issued_par >> q & 1u, nullptr);
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+                const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+                const int buf = it & 1;
+                const uint32_t aph = (it >> 1) & 1;
+                if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem_base + buf * BN;
+                const uint32_t idesc = idesc_bf16(128, tl.n);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
+                    tc_fence_after();
+                    if (MODE != kDown) fence_proxy_async_smem();   // cp.async-written rows -> tensor core
+                    const uint64_t ad = sdesc_sw128(smem_u32(sA + size_t(s) * kAStage));
+                    const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                    umma_commit(&empty[s]);
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit(&tfull[buf]);
+            }
+            if (!ok) {
+                report_error(g.err, kErrWaitExpired);
+                *s_abort = 1;
+            }
+            // all MMAs issued by this thread complete before TMEM is freed
+            umma_commit(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        // The four warps run the same tile sequence and the same named
+        // barriers; after an abort they keep looping without touching TMEM or
+        // global memory, so no warp is left waiting at a barrier.
+        const int sub = warp & 3;                 // TMEM lane quarter this warp may access
+        const int lrow = 32 * sub + lane;         // row of the 128-row tile
+        const int et = threadIdx.x - 64;          // 0..127
+        int it = 0;
+        bool dead = false;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const int buf = it & 1;
+            const uint32_t aph = (it >> 1) & 1;
+            if (MODE == kDown) {
+                for (int c = et; c < tl.ntok; c += 128) {
+                    const int p = g.perm[tl.row0 + c];
+                    s_tok[c] = p / g.k;
+                    s_tokw[c] = g.topk_w[p];
+                }
+                named_bar(1, 128);
+            }
+            if (!dead) {
+                const bool ok = mbar_wait(&tfull[buf], aph, s_abort);
+                if (__any_sync(0xffffffffu, !ok)) {     // warp-uniform: tcgen05.ld is warp-collective
+                    if (lane == 0) report_error(g.err, kErrWaitExpired);
+                    *s_abort = 1;
+                    dead = true;
+                }
+            }
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + (uint32_t(32 * sub) << 16) + buf * BN;
+            for (int c0 = 0; c0 < tl.n; c0 += 16) {
+                float v[16];
+                if (dead) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                } else {
+                    tmem_ld16(tbase + c0, v);
+                }
+                if (MODE == kDown) {
+                    const int f = tl.wt * 128 + lrow;
+                    if (!dead && f < g.feats) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = c0 + i;
+                            if (c < tl.ntok) red_add_f32(g.y_acc + (size_t)s_tok[c] * g.H + f, s_tokw[c] * v[i]);
+                        }
+                    }
+                } else if (MODE == kUpRelu2) {
+                    const int f = tl.wt * 128 + lrow;
+                    if (!dead && f < g.feats) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = c0 + i;
+                            if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_relu2(v[i]));
+                        }
+                    }
+                } else {
+                    // up rows (lanes 64..127) hand their values to the gate rows through shared memory
+                    if (sub >= 2) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) s_u[(lrow - 64) * 17 + i] = v[i];
+                    }
+                    named_bar(1, 128);
+                    if (!dead && sub < 2) {
+                        const int f = tl.wt * 64 + lrow;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = c0 + i;
+                            if (c < tl.ntok)
+                                g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_swiglu(v[i], s_u[lrow * 17 + i]));
+                        }
+                    }
+                    named_bar(1, 128);
+                }
+            }
+            tc_fence_before();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (MODE == kDown) named_bar(1, 128);   // s_tok reuse
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+    pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------- host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 matrix (outer rows x inner cols, row-major), 128-byte swizzled boxes.
+cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                      uint32_t box_outer) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE, int BN, int STAGES>
+cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, bool pdl, cudaStream_t s) {
+    CUtensorMap tA, tB;
+    const uint32_t a_box = MODE == kUpSwiglu ? 64 : 128;
+    cudaError_t e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E * g.rows_per_expert, kBK, a_box);
+    if (e != cudaSuccess) return e;
+    if (MODE == kDown) {
+        e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, 16);
+    } else {
+        e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);   // unused by the up kernels
+    }
+    if (e != cudaSuccess) return e;
+    auto kern = k_gemm<MODE, BN, STAGES>;
+    const size_t smem = Smem<BN, STAGES>::kBytes;
+    if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+    return launch_k(kern, dim3(device_info().sm_count), dim3(kThreads), smem, s, pdl, tA, tB, g);
+}
+
+// Token-tile width from the mean pairs per expert.
+int pick_bn(const ExpertArgs& a) {
+    const double mean = (double)a.T * a.k / a.E;
+    if (mean <= 24.0) return 32;
+    if (mean <= 96.0) return 128;
+    return 256;
+}
+
+GemmParams params(const ExpertArgs& a, bool up) {
+    GemmParams g{};
+    g.counts = a.counts;
+    g.offsets = a.offsets;
+    g.perm = a.perm;
+    g.topk_w = a.topk_w;
+    g.x = a.x;
+    g.h = a.h;
+    g.y_acc = a.y_acc;
+    g.E = a.E;
+    g.k = a.k;
+    g.H = a.H;
+    g.I = a.I;
+    g.err = a.err;
+    if (up) {
+        g.K = a.H;
+        g.rows_per_expert = a.act == 0 ? 2 * a.I : a.I;
+        g.feats = a.I;
+    } else {
+        g.K = a.I;
+        g.rows_per_expert = a.H;
+        g.feats = a.H;
+    }
+    return g;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
+    if (a.fmt != 0) return cudaErrorNotSupported;
+    const GemmParams g = params(a, true);
+    const int bn = pick_bn(a);
+    if (a.act == 0) {
+        if (bn == 32) return run<kUpSwiglu, 32, 8>(a, g, a.w1, pdl, s);
+        if (bn == 128) return run<kUpSwiglu, 128, 5>(a, g, a.w1, pdl, s);
+        return run<kUpSwiglu, 256, 4>(a, g, a.w1, pdl, s);
+    }
+    if (bn == 32) return run<kUpRelu2, 32, 8>(a, g, a.w1, pdl, s);
+    if (bn == 128) return run<kUpRelu2, 128, 5>(a, g, a.w1, pdl, s);
+    return run<kUpRelu2, 256, 4>(a, g, a.w1, pdl, s);
+}
+
+cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
+    if (a.fmt != 0) return cudaErrorNotSupported;
+    const GemmParams g = params(a, false);
+    const int bn = pick_bn(a);
+    if (bn == 32) return run<kDown, 32, 8>(a, g, a.w2, pdl, s);
+    if (bn == 128) return run<kDown, 128, 5>(a, g, a.w2, pdl, s);
+    return run<kDown, 256, 4>(a, g, a.w2, pdl, s);
+}
 
 }  // namespace moe
