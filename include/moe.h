@@ -74,9 +74,9 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1 } moe_wfmt;
 
 /* Which expert kernels moe_experts / moe_forward use (process-wide). */
 typedef enum {
-    MOE_DISPATCH_AUTO = 0, /* grouped GEMV when T <= 64, tcgen05 grouped GEMM above */
-    MOE_DISPATCH_GEMV = 1, /* always the weight-streaming grouped GEMV */
-    MOE_DISPATCH_GEMM = 2  /* always the tcgen05 grouped GEMM */
+    MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM at every T */
+    MOE_DISPATCH_GEMV = 1, /* the CUDA-core weight-streaming grouped GEMV (bf16 only) */
+    MOE_DISPATCH_GEMM = 2  /* the tcgen05 grouped GEMM */
 } moe_dispatch;
 
 /* Problem sizes.  T tokens, H hidden, E experts, k picks per token, I expert
@@ -130,7 +130,7 @@ typedef struct {
 typedef struct {
     size_t y_acc;   /* fp32 (T, H): the unscaled routed sum */
     size_t h;       /* bf16 (P, I): activations in plan order */
-    size_t xs;      /* bf16 (P, H): x rows gathered in plan order (GEMM path) */
+    size_t xs;      /* bf16 (P, H): token rows gathered in plan order (wide token tiles) */
     size_t scratch; /* plan and scheduler scratch */
     size_t total;   /* == moe_workspace_bytes() */
 } moe_ws_layout;

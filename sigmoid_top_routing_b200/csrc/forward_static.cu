@@ -153,8 +153,9 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
         p.inv = plan->inv;
         p.tiles = plan->tiles;
         p.err = err;
-        if ((e = launch_plan(p, true, s)) != cudaSuccess) return cuda_fail(e, "plan");
-        ++launched;
+        int np = 0;   // no scratch given: the single-CTA plan
+        if ((e = launch_plan(p, true, s, &np)) != cudaSuccess) return cuda_fail(e, "plan");
+        launched += np;
     }
     ExpertArgs a{};
     a.x = static_cast<const uint16_t*>(x);

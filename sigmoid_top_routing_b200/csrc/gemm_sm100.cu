@@ -76,7 +76,8 @@ struct Smem {
     static constexpr size_t kTok = kTileBase + 257 * 4;                       // BN ints (token of column)
     static constexpr size_t kTokW = kTok + BN * 4;                            // BN floats
     static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats
-    static constexpr size_t kEnd = kU + 64 * 17 * 4;
+    static constexpr size_t kTrow = kU + 64 * 17 * 4;                         // BN ints (producer's token rows)
+    static constexpr size_t kEnd = kTrow + BN * 4;
     static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
 };
 
@@ -135,11 +136,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_tok = reinterpret_cast<int*>(sm + L::kTok);
     float* s_tokw = reinterpret_cast<float*>(sm + L::kTokW);
     float* s_u = reinterpret_cast<float*>(sm + L::kU);
+    int* s_trow = reinterpret_cast<int*>(sm + L::kTrow);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
     // up: 32 producer lanes gather token rows with cp.async, + 1 expect_tx arrive
-    constexpr uint32_t kFullCount = MODE == kDown ? 1 : 33;
+    // decode-width up tiles gather token rows from x with cp.async (32 lanes + the
+    // expect_tx arrive); wider tiles take rows of xs (up) or h (down) by TMA
+    constexpr bool kGather = MODE != kDown && BN <= 32;
+    constexpr uint32_t kFullCount = kGather ? 33 : 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -156,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
-        if (MODE == kDown) tma_prefetch_desc(&tmB);
+        if (!kGather) tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, kTmemCols);
@@ -203,52 +208,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t issued_mask = 0;            // stages with a fill whose arrival is not yet known
         uint32_t issued_par = 0;             // parity of that fill
         bool ok = true;
+        // weights read by one token tile are streamed once (evict first); with
+        // several token tiles per weight tile the neighbours re-read it from L2
         const uint64_t pol_w = policy_evict_first();
+        const bool hint_w = BN <= 32;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
-            // token rows of this tile (up: gathered from x by pair)
-            const uint16_t* trow[BN / 32 > 0 ? BN / 32 : 1];
-            if (MODE != kDown) {
-#pragma unroll
-                for (int j = 0; j < (BN + 31) / 32; ++j) {
-                    const int r = lane + 32 * j;
-                    const int rr = r < tl.ntok ? r : (tl.ntok - 1);   // pad with a valid row
-                    const int p = g.perm[tl.row0 + rr];
-                    trow[j] = g.x + (size_t)(p / g.k) * g.H;
+            if (kGather) {
+                // token row of each B row (padding rows repeat the last token)
+                __syncwarp();
+                for (int r = lane; r < tl.n; r += 32) {
+                    const int rr = r < tl.ntok ? r : tl.ntok - 1;
+                    s_trow[r] = g.perm[tl.row0 + rr] / g.k;
                 }
+                __syncwarp();
             }
             const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
             for (int kb = 0; kb < nkb; ++kb) {
-                if (!mbar_wait(&empty[s], ph ^ 1, s_abort)) { ok = false; break; }
+                // all 32 lanes wait on the same phase; the decision is made warp-uniform
+                const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 if (lane == 0) {
-                    const uint32_t bytes = kAStage + (MODE == kDown ? tl.n * 128 : 0);
+                    const uint32_t bytes = kAStage + (kGather ? 0 : tl.n * 128);
                     mbar_arrive_expect_tx(&full[s], bytes);
                     unsigned char* a = sA + size_t(s) * kAStage;
-                    if (MODE == kUpSwiglu) {
+                    if (hint_w) {
                         tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
-                        tma_load_2d_hint(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s], pol_w);
+                        if (MODE == kUpSwiglu)
+                            tma_load_2d_hint(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s], pol_w);
                     } else {
-                        tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
+                        tma_load_2d(a, &tmA, kb * kBK, a_row, &full[s]);
+                        if (MODE == kUpSwiglu) tma_load_2d(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s]);
                     }
-                    if (MODE == kDown) {
+                    if (!kGather) {
                         unsigned char* b = sB + size_t(s) * L::kBStage;
                         for (int j = 0; j < tl.n / 16; ++j)
                             tma_load_2d(b + j * 2048, &tmB, kb * kBK, tl.row0 + 16 * j, &full[s]);
                     }
                 }
-                if (MODE != kDown) {
-                    // gather: row r, 16-byte chunk c -> swizzled (r, c ^ (r & 7))
+                if (kGather) {
+                    // gather: 8 lanes cover one 128-byte row slice, 4 rows per instruction;
+                    // row r, 16-byte chunk c lands at the swizzled (r, c ^ (r & 7))
                     const uint32_t b = smem_u32(sB + size_t(s) * L::kBStage);
-#pragma unroll
-                    for (int j = 0; j < (BN + 31) / 32; ++j) {
-                        const int r = lane + 32 * j;
-                        if (r < tl.n) {
-                            const unsigned char* src = reinterpret_cast<const unsigned char*>(trow[j]) + kb * 128;
-#pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                cp_async16(b + r * 128 + ((c ^ (r & 7)) << 4), src + c * 16);
-                        }
-                    }
+                    const int c = lane & 7;
+                    const unsigned char* xb = reinterpret_cast<const unsigned char*>(g.x) + kb * 128 + c * 16;
+                    for (int r = lane >> 3; r < tl.n; r += 4)
+                        cp_async16(b + r * 128 + ((c ^ (r & 7)) << 4), xb + (size_t)s_trow[r] * g.H * 2);
                     cp_async_arrive(&full[s]);
                 }
                 issued_mask |= 1u << s;
@@ -281,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    if (MODE != kDown) fence_proxy_async_smem();   // cp.async-written rows -> tensor core
+                    if (kGather) fence_proxy_async_smem();   // cp.async-written rows -> tensor core
                     const uint64_t ad = sdesc_sw128(smem_u32(sA + size_t(s) * kAStage));
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
 #pragma unroll
@@ -435,8 +440,10 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
         e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, 16);
+    } else if (BN > 32) {
+        e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, 16);   // rows gathered in plan order
     } else {
-        e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);   // unused by the up kernels
+        e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);          // unused (cp.async gather)
     }
     if (e != cudaSuccess) return e;
     auto kern = k_gemm<MODE, BN, STAGES>;
@@ -479,7 +486,30 @@ GemmParams params(const ExpertArgs& a, bool up) {
     return g;
 }
 
+// xs[pos] = x[perm[pos] / k]: token rows in plan order, one warp per row.
+__global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+                                                     uint16_t* __restrict__ xs, int P, int k, int H) {
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n16 = H / 8;
+    for (int pos = blockIdx.x * 8 + warp; pos < P; pos += gridDim.x * 8) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(perm[pos] / k) * H);
+        uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)pos * H);
+        for (int c = lane; c < n16; c += 32) dst[c] = ld_nc(src + c);
+    }
+    pdl_trigger();
+}
+
 }  // namespace
+
+bool gemm_needs_xs(const ExpertArgs& a) { return a.fmt == 0 && pick_bn(a) > 32; }
+
+cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
+    const int P = a.T * a.k;
+    if (P == 0) return cudaSuccess;
+    const int blocks = min((P + 7) / 8, device_info().sm_count * 16);
+    return launch_k(k_gather_rows, dim3(blocks), dim3(256), 0, s, pdl, a.x, a.perm, a.xs, P, a.k, a.H);
+}
 
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     if (a.fmt != 0) return cudaErrorNotSupported;

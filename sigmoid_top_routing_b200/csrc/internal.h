@@ -30,6 +30,7 @@ struct PlanArgs {
     const int32_t* idx;
     int P, E, k;
     int32_t *counts, *offsets, *perm, *inv, *tiles;
+    int32_t* scratch;        // plan_scratch_ints(P, E) ints for the multi-CTA plan, or null
     int* err;
 };
 
@@ -68,12 +69,18 @@ const DeviceInfo& device_info();   // of the current device (cached)
 // Launchers: return the first CUDA error, cudaSuccess otherwise.
 // launch_route sets *n_launched to the number of kernels it enqueued.
 cudaError_t launch_route(const RouteArgs& a, bool fuse_plan, bool pdl, cudaStream_t s, int* n_launched);
-cudaError_t launch_plan(const PlanArgs& a, bool pdl, cudaStream_t s);
+// launch_plan sets *n_launched to the number of kernels it enqueued (1 or 3).
+cudaError_t launch_plan(const PlanArgs& a, bool pdl, cudaStream_t s, int* n_launched);
+size_t plan_scratch_ints(int P, int E);
 cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // The tcgen05 grouped GEMMs (cudaErrorNotSupported where a format has none).
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// Wide token tiles take the up GEMM's token rows from xs (plan order), filled
+// by launch_gather_x; decode-width tiles gather from x themselves.
+bool gemm_needs_xs(const ExpertArgs& a);
+cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s);
 

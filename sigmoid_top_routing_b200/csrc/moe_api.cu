@@ -48,9 +48,6 @@ thread_local Hook g_hook;
 std::mutex g_dispatch_mu;
 int g_dispatch = MOE_DISPATCH_AUTO;
 
-// Token counts up to this use the weight-streaming GEMV under MOE_DISPATCH_AUTO.
-constexpr int kGemvMaxT = 64;
-
 moe_status fail(moe_status st, const char* fmt, ...) {
     char buf[512];
     va_list ap;
@@ -95,10 +92,10 @@ void layout(const moe_dims* d, moe_ws_layout* L) {
     off = align256(off + T * H * 4);
     L->h = off;
     off = align256(off + P * I * 2);
-    L->xs = off;
+    L->xs = off;          // token rows gathered in plan order (wide token tiles)
     off = align256(off + P * H * 2);
-    L->scratch = off;
-    off = align256(off + (size_t)kSmallT * E * 4 + 4096);
+    L->scratch = off;     // router logits (T <= 32) | multi-CTA plan histograms and bases
+    off = align256(off + (size_t)kSmallT * E * 4 + 4096 + plan_scratch_ints((int)P, (int)E) * 4);
     L->total = off;
 }
 
@@ -107,6 +104,7 @@ struct WsView {
     uint16_t* h;
     uint16_t* xs;
     float* l_scratch;
+    int32_t* plan_scratch;
 };
 
 moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
@@ -121,6 +119,7 @@ moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
     v->h = reinterpret_cast<uint16_t*>(b + L.h);
     v->xs = reinterpret_cast<uint16_t*>(b + L.xs);
     v->l_scratch = reinterpret_cast<float*>(b + L.scratch);
+    v->plan_scratch = reinterpret_cast<int32_t*>(b + L.scratch + (size_t)kSmallT * d->E * 4 + 4096);
     return MOE_OK;
 }
 
@@ -166,12 +165,9 @@ int current_dispatch() {
     return g_dispatch;
 }
 
-bool use_gemv(const moe_dims* d) {
-    const int mode = current_dispatch();
-    if (mode == MOE_DISPATCH_GEMV) return true;
-    if (mode == MOE_DISPATCH_GEMM) return false;
-    return d->T <= kGemvMaxT;
-}
+// The tcgen05 grouped GEMM serves every token count (its token tiles shrink
+// to N = 16 for decode batches); the CUDA-core GEMV stays selectable.
+bool use_gemv(const moe_dims*) { return current_dispatch() == MOE_DISPATCH_GEMV; }
 
 ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* topk_w,
                             const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
@@ -238,7 +234,13 @@ struct Seq {
 
 moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
     const bool gemv = use_gemv(d);
-    cudaError_t e = q.stage(MOE_STAGE_UP, [&](int*) {
+    cudaError_t e;
+    if (!gemv && gemm_needs_xs(a)) {
+        // token rows in plan order for the wide up tiles (part of the plan's data movement)
+        e = q.stage(-1, [&](int*) { return launch_gather_x(a, true, q.s); });
+        if (e != cudaSuccess) return cuda_fail(e, "gather token rows");
+    }
+    e = q.stage(MOE_STAGE_UP, [&](int*) {
         return gemv ? launch_gemv_up(a, true, q.s) : launch_gemm_up(a, true, q.s);
     });
     if (e == cudaErrorNotSupported)
@@ -255,8 +257,9 @@ moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
     return MOE_OK;
 }
 
-PlanArgs make_plan_args(const int32_t* idx, const moe_dims* d, const moe_plan_t* plan) {
+PlanArgs make_plan_args(const int32_t* idx, const moe_dims* d, const moe_plan_t* plan, int32_t* scratch) {
     PlanArgs p{};
+    p.scratch = scratch;
     p.idx = idx;
     p.P = d->T * d->k;
     p.E = d->E;
@@ -333,9 +336,9 @@ moe_status moe_plan(const int32_t* topk_idx, const moe_dims* d, const moe_plan_t
     if ((st = check_plan(plan)) != MOE_OK) return st;
     WsView v;
     if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
-    const PlanArgs p = make_plan_args(topk_idx, d, plan);
+    const PlanArgs p = make_plan_args(topk_idx, d, plan, v.plan_scratch);
     Seq q{reinterpret_cast<cudaStream_t>(stream)};
-    cudaError_t e = q.stage(MOE_STAGE_PLAN, [&](int*) { return launch_plan(p, true, q.s); });
+    cudaError_t e = q.stage(MOE_STAGE_PLAN, [&](int* n) { return launch_plan(p, true, q.s, n); });
     if (e != cudaSuccess) return cuda_fail(e, "plan");
     g_launches = q.n;
     return MOE_OK;
@@ -408,8 +411,8 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
     cudaError_t e = q.stage(MOE_STAGE_ROUTE, [&](int* n) { return launch_route(r, fuse, true, q.s, n); });
     if (e != cudaSuccess) return cuda_fail(e, "route");
     if (!fuse) {
-        const PlanArgs p = make_plan_args(topk_idx, d, plan);
-        e = q.stage(MOE_STAGE_PLAN, [&](int*) { return launch_plan(p, true, q.s); });
+        const PlanArgs p = make_plan_args(topk_idx, d, plan, v.plan_scratch);
+        e = q.stage(MOE_STAGE_PLAN, [&](int* n) { return launch_plan(p, true, q.s, n); });
         if (e != cudaSuccess) return cuda_fail(e, "plan");
     }
     const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);

@@ -198,102 +198,127 @@ __global__ void __launch_bounds__(256) k_select(RouteArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Large T: TT tokens per CTA.  Warp w computes segment w for all TT tokens
-// and all experts (lane holds experts lane + 32 i), staging the router chunk
-// (transposed) and the token chunk (fp32) in its own shared memory; then the
-// 8 partials are summed in order and each warp selects for TT / 8 tokens.
+// Large T: TT tokens per CTA.  Warp w computes segment w (the canonical order)
+// for all TT tokens and all EP = 32 NE experts as a register-blocked
+// micro-GEMM: lane (tg = lane % 8, eg = lane / 8) owns tokens tg TPT .. and
+// experts eg EPT .. (TPT = TT / 8, EPT = EP / 4), so each h costs 1-2 shared
+// loads of token values and EPT / 4 of router values for TPT x EPT FMAs.
+// Every (token, expert) logit is still one fmaf chain over the segment in
+// increasing h, so the bits equal the small-T kernel's.  For E <= 64 the next
+// chunk's router and token values are loaded into registers while the
+// current chunk is computed.
 template <int NE, int TT, int HCH>
 __global__ void __launch_bounds__(256) k_route_large(RouteArgs a) {
     extern __shared__ float sm[];
-    constexpr int EP = 32 * NE;
+    constexpr int EP = 32 * NE, TPT = TT / 8, EPT = EP / 4;
     constexpr int WARP_FLOATS = HCH * EP + HCH * TT;
+    constexpr bool PF = NE <= 2;                  // register prefetch of the next chunk
+    constexpr int WV = HCH / 4;                   // float4 of router values per expert per chunk
+    constexpr int XV = HCH / 8;                   // uint4 of token values per token per chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tg = lane & 7, eg = lane >> 3;
     float* wt = sm + warp * WARP_FLOATS;          // [HCH][EP]
     float* xs = wt + HCH * EP;                    // [HCH][TT]
     pdl_wait();
     zero_slice(a);
     const int t0 = blockIdx.x * TT;
     const int E = a.E, H = a.H;
+    const int nsub = H / HCH;                     // staging pieces along h
+    constexpr int kPer = kChunk / HCH;            // pieces per canonical chunk
 
-    float acc[TT][NE];
+    float acc[TPT][EPT];
 #pragma unroll
-    for (int m = 0; m < TT; ++m)
+    for (int i = 0; i < TPT; ++i)
 #pragma unroll
-        for (int i = 0; i < NE; ++i) acc[m][i] = 0.0f;
+        for (int j = 0; j < EPT; ++j) acc[i][j] = 0.0f;
 
-    for (int c = warp; c < H / kChunk; c += kSegs) {
+    float4 rw[NE][WV];
+    uint4 rx[XV];
+    // piece q of this warp's segment: canonical chunk warp + 8 (q / kPer), part q % kPer
+    auto piece_h0 = [&](int q) { return (warp + kSegs * (q / kPer)) * kChunk + (q % kPer) * HCH; };
+    const int npieces = ((H / kChunk - warp + kSegs - 1) / kSegs) * kPer;
+    auto load = [&](int q) {
+        const int h0 = piece_h0(q);
 #pragma unroll
-        for (int half = 0; half < kChunk / HCH; ++half) {
-            const int h0 = c * kChunk + half * HCH;
-            // stage router chunk transposed: wt[hh][e]
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+            const float4* src = reinterpret_cast<const float4*>(a.w_router + (size_t)(e < E ? e : 0) * H + h0);
 #pragma unroll
-            for (int i = 0; i < NE; ++i) {
-                const int e = lane + 32 * i;
-                if (e < E) {
-                    const float4* src = reinterpret_cast<const float4*>(a.w_router + (size_t)e * H + h0);
-#pragma unroll
-                    for (int q = 0; q < HCH / 4; ++q) {
-                        const float4 v = __ldg(src + q);
-                        wt[(4 * q + 0) * EP + e] = v.x;
-                        wt[(4 * q + 1) * EP + e] = v.y;
-                        wt[(4 * q + 2) * EP + e] = v.z;
-                        wt[(4 * q + 3) * EP + e] = v.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int hh = 0; hh < HCH; ++hh) wt[hh * EP + e] = 0.0f;
-                }
-            }
-            // stage token chunk: xs[hh][t]
-            if (lane < TT) {
-                const int t = t0 + lane;
-                if (t < a.T) {
-                    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * H + h0);
-#pragma unroll
-                    for (int q = 0; q < HCH / 8; ++q) {
-                        const uint4 v = ld_nc(src + q);
-                        xs[(8 * q + 0) * TT + lane] = bf16lo(v.x);
-                        xs[(8 * q + 1) * TT + lane] = bf16hi(v.x);
-                        xs[(8 * q + 2) * TT + lane] = bf16lo(v.y);
-                        xs[(8 * q + 3) * TT + lane] = bf16hi(v.y);
-                        xs[(8 * q + 4) * TT + lane] = bf16lo(v.z);
-                        xs[(8 * q + 5) * TT + lane] = bf16hi(v.z);
-                        xs[(8 * q + 6) * TT + lane] = bf16lo(v.w);
-                        xs[(8 * q + 7) * TT + lane] = bf16hi(v.w);
-                    }
-                } else {
-#pragma unroll
-                    for (int hh = 0; hh < HCH; ++hh) xs[hh * TT + lane] = 0.0f;
-                }
-            }
-            __syncwarp();
-#pragma unroll 4
-            for (int hh = 0; hh < HCH; ++hh) {
-                float wv[NE];
-#pragma unroll
-                for (int i = 0; i < NE; ++i) wv[i] = wt[hh * EP + lane + 32 * i];
-                const float4* x4 = reinterpret_cast<const float4*>(xs + hh * TT);
-#pragma unroll
-                for (int m4 = 0; m4 < TT / 4; ++m4) {
-                    const float4 xv = x4[m4];
-#pragma unroll
-                    for (int i = 0; i < NE; ++i) {
-                        acc[4 * m4 + 0][i] = fmaf(xv.x, wv[i], acc[4 * m4 + 0][i]);
-                        acc[4 * m4 + 1][i] = fmaf(xv.y, wv[i], acc[4 * m4 + 1][i]);
-                        acc[4 * m4 + 2][i] = fmaf(xv.z, wv[i], acc[4 * m4 + 2][i]);
-                        acc[4 * m4 + 3][i] = fmaf(xv.w, wv[i], acc[4 * m4 + 3][i]);
-                    }
-                }
-            }
-            __syncwarp();
+            for (int v = 0; v < WV; ++v) rw[i][v] = e < E ? __ldg(src + v) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        const int t = t0 + lane;
+        const bool tv = lane < TT && t < a.T;
+        const uint4* xsrc = reinterpret_cast<const uint4*>(a.x + (size_t)(tv ? t : 0) * H + h0);
+#pragma unroll
+        for (int v = 0; v < XV; ++v) rx[v] = tv ? ld_nc(xsrc + v) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto stage = [&]() {
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            const int e = lane + 32 * i;
+#pragma unroll
+            for (int v = 0; v < WV; ++v) {
+                wt[(4 * v + 0) * EP + e] = rw[i][v].x;
+                wt[(4 * v + 1) * EP + e] = rw[i][v].y;
+                wt[(4 * v + 2) * EP + e] = rw[i][v].z;
+                wt[(4 * v + 3) * EP + e] = rw[i][v].w;
+            }
+        }
+        if (lane < TT) {
+#pragma unroll
+            for (int v = 0; v < XV; ++v) {
+                xs[(8 * v + 0) * TT + lane] = bf16lo(rx[v].x);
+                xs[(8 * v + 1) * TT + lane] = bf16hi(rx[v].x);
+                xs[(8 * v + 2) * TT + lane] = bf16lo(rx[v].y);
+                xs[(8 * v + 3) * TT + lane] = bf16hi(rx[v].y);
+                xs[(8 * v + 4) * TT + lane] = bf16lo(rx[v].z);
+                xs[(8 * v + 5) * TT + lane] = bf16hi(rx[v].z);
+                xs[(8 * v + 6) * TT + lane] = bf16lo(rx[v].w);
+                xs[(8 * v + 7) * TT + lane] = bf16hi(rx[v].w);
+            }
+        }
+    };
+    (void)nsub;
+    if (PF && npieces > 0) load(0);
+    for (int q = 0; q < npieces; ++q) {
+        if (!PF) load(q);
+        stage();
+        __syncwarp();
+        if (PF && q + 1 < npieces) load(q + 1);
+#pragma unroll 4
+        for (int hh = 0; hh < HCH; ++hh) {
+            float xv[TPT];
+            const float* xr = xs + hh * TT + tg * TPT;
+            if (TPT == 4) {
+                const float4 t4 = *reinterpret_cast<const float4*>(xr);
+                xv[0] = t4.x; xv[TPT > 1 ? 1 : 0] = t4.y; xv[TPT > 2 ? 2 : 0] = t4.z; xv[TPT > 3 ? 3 : 0] = t4.w;
+            } else if (TPT == 2) {
+                const float2 t2 = *reinterpret_cast<const float2*>(xr);
+                xv[0] = t2.x; xv[TPT > 1 ? 1 : 0] = t2.y;
+            } else {
+                xv[0] = xr[0];
+            }
+            const float4* wr = reinterpret_cast<const float4*>(wt + hh * EP + eg * EPT);
+#pragma unroll
+            for (int v = 0; v < EPT / 4; ++v) {
+                const float4 w4 = wr[v];
+#pragma unroll
+                for (int i = 0; i < TPT; ++i) {
+                    acc[i][4 * v + 0] = fmaf(xv[i], w4.x, acc[i][4 * v + 0]);
+                    acc[i][4 * v + 1] = fmaf(xv[i], w4.y, acc[i][4 * v + 1]);
+                    acc[i][4 * v + 2] = fmaf(xv[i], w4.z, acc[i][4 * v + 2]);
+                    acc[i][4 * v + 3] = fmaf(xv[i], w4.w, acc[i][4 * v + 3]);
+                }
+            }
+        }
+        __syncwarp();
     }
     __syncthreads();
     float* part = sm;                              // [8][TT][EP]
 #pragma unroll
-    for (int m = 0; m < TT; ++m)
+    for (int i = 0; i < TPT; ++i)
 #pragma unroll
-        for (int i = 0; i < NE; ++i) part[(warp * TT + m) * EP + lane + 32 * i] = acc[m][i];
+        for (int j = 0; j < EPT; ++j) part[(warp * TT + tg * TPT + i) * EP + eg * EPT + j] = acc[i][j];
     __syncthreads();
     for (int m = warp; m < TT; m += kSegs) {
         const int t = t0 + m;
