@@ -44,7 +44,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kBK = 64;                  // k per stage: 64 bf16 = one 128-byte swizzle row
-constexpr int kAStage = 128 * kBK * 2;   // 16 KB of weight rows per stage
+constexpr int kARows = 128 * kBK * 2;    // 16 KB: 128 weight rows of one k-block
 constexpr int kThreads = 192;
 
 enum Mode { kUpSwiglu = 0, kUpRelu2 = 1, kDown = 2 };
@@ -64,11 +64,11 @@ struct GemmParams {
     int* err;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int ASTAGE>
 struct Smem {
     static constexpr int kBStage = BN * 128;
     static constexpr size_t kA = 0;
-    static constexpr size_t kB = kA + size_t(STAGES) * kAStage;
+    static constexpr size_t kB = kA + size_t(STAGES) * ASTAGE;
     static constexpr size_t kBar = kB + size_t(STAGES) * kBStage;           // 8-byte barriers
     static constexpr int kNumBar = 2 * STAGES + 4 + 1;                      // full, empty, tfull[2], tempty[2], drain
     static constexpr size_t kMisc = kBar + kNumBar * 8;                       // tmem base, abort flag
@@ -109,6 +109,10 @@ MOE_DEV Tile decode_tile(int t, const int* base, int E, const int32_t* counts, c
     return r;
 }
 
+// silu(g) * u in fp32 with the fast exponential and division (the result is
+// rounded to bf16); NaN propagates, g -> -inf gives -0 * u.
+MOE_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
+
 MOE_DEV void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -119,7 +123,14 @@ MOE_DEV void cp_async_arrive(uint64_t* bar) {
 template <int MODE, int BN, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams g) {
-    using L = Smem<BN, STAGES>;
+    // SwiGLU with wide token tiles keeps two accumulators (128 gate rows and
+    // 128 up rows against one token tile) so a thread holds gate and up of its
+    // feature; decode-width SwiGLU tiles split 64 gate + 64 up rows over the
+    // lanes of one accumulator (more, smaller tiles for a short decode step).
+    constexpr bool kDual = MODE == kUpSwiglu && BN >= 64;
+    constexpr int kAStage = kDual ? 2 * kARows : kARows;
+    constexpr int kBoxRows = BN < 64 ? 16 : 64;       // token rows per TMA box
+    using L = Smem<BN, STAGES, kAStage>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sA = sm + L::kA;
@@ -139,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_trow = reinterpret_cast<int*>(sm + L::kTrow);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+    constexpr uint32_t kTmemCols = (kDual ? 4 : 2) * BN < 32 ? 32 : (kDual ? 4 : 2) * BN;
     // up: 32 producer lanes gather token rows with cp.async, + 1 expect_tx arrive
     // decode-width up tiles gather token rows from x with cp.async (32 lanes + the
     // expect_tx arrive); wider tiles take rows of xs (up) or h (down) by TMA
@@ -170,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     pdl_wait();   // the plan and (for down) h come from earlier kernels
     // tile table: tiles of expert e = weight tiles x ceil(count / BN)
-    const int fpt = MODE == kUpSwiglu ? 64 : 128;      // output features per tile
+    const int fpt = (MODE == kUpSwiglu && !kDual) ? 64 : 128;   // output features per tile
     const int n_wt = (g.feats + fpt - 1) / fpt;
     if (warp == 2) {
         const int per = (g.E + 31) / 32;
@@ -229,9 +240,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 if (lane == 0) {
-                    const uint32_t bytes = kAStage + (kGather ? 0 : tl.n * 128);
+                    const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
+                    const uint32_t bytes = kAStage + (kGather ? 0 : nbox * kBoxRows * 128);
                     mbar_arrive_expect_tx(&full[s], bytes);
                     unsigned char* a = sA + size_t(s) * kAStage;
+                    // A: [gate | up] halves for SwiGLU (64 or 128 rows each), else 128 rows
                     if (hint_w) {
                         tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
                         if (MODE == kUpSwiglu)
@@ -242,8 +255,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!kGather) {
                         unsigned char* b = sB + size_t(s) * L::kBStage;
-                        for (int j = 0; j < tl.n / 16; ++j)
-                            tma_load_2d(b + j * 2048, &tmB, kb * kBK, tl.row0 + 16 * j, &full[s]);
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
                     }
                 }
                 if (kGather) {
@@ -281,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d = tmem_base + buf * BN;
+                const uint32_t d = tmem_base + buf * (kDual ? 2 * BN : BN);
                 const uint32_t idesc = idesc_bf16(128, tl.n);
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
@@ -290,8 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t ad = sdesc_sw128(smem_u32(sA + size_t(s) * kAStage));
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
                         umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                        if (kDual)   // up rows: the second 16 KB of the A stage, accumulator at + BN columns
+                            umma_bf16(d + BN, ad + uint64_t((kARows >> 4) + kk * 2), bd + uint64_t(kk * 2), idesc,
+                                      (kb | kk) != 0);
+                    }
                     umma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
                 }
@@ -338,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tc_fence_after();
-            const uint32_t tbase = tmem_base + (uint32_t(32 * sub) << 16) + buf * BN;
+            const uint32_t tbase = tmem_base + (uint32_t(32 * sub) << 16) + buf * (kDual ? 2 * BN : BN);
             for (int c0 = 0; c0 < tl.n; c0 += 16) {
                 float v[16];
                 if (dead) {
@@ -365,6 +382,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_relu2(v[i]));
                         }
                     }
+                } else if (kDual) {
+                    float u[16];
+                    if (dead) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) u[i] = 0.0f;
+                    } else {
+                        tmem_ld16(tbase + BN + c0, u);
+                    }
+                    const int f = tl.wt * 128 + lrow;
+                    if (!dead && f < g.feats) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int c = c0 + i;
+                            if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(v[i], u[i]));
+                        }
+                    }
                 } else {
                     // up rows (lanes 64..127) hand their values to the gate rows through shared memory
                     if (sub >= 2) {
@@ -378,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
                             if (c < tl.ntok)
-                                g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_swiglu(v[i], s_u[lrow * 17 + i]));
+                                g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(v[i], s_u[lrow * 17 + i]));
                         }
                     }
                     named_bar(1, 128);
@@ -435,19 +468,21 @@ cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
 template <int MODE, int BN, int STAGES>
 cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, bool pdl, cudaStream_t s) {
     CUtensorMap tA, tB;
-    const uint32_t a_box = MODE == kUpSwiglu ? 64 : 128;
+    const uint32_t a_box = (MODE == kUpSwiglu && BN < 64) ? 64 : 128;
+    const uint32_t b_box = BN < 64 ? 16 : 64;
     cudaError_t e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E * g.rows_per_expert, kBK, a_box);
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
-        e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, 16);
+        e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, b_box);
     } else if (BN > 32) {
-        e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, 16);   // rows gathered in plan order
+        e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, b_box);   // rows gathered in plan order
     } else {
         e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);          // unused (cp.async gather)
     }
     if (e != cudaSuccess) return e;
     auto kern = k_gemm<MODE, BN, STAGES>;
-    const size_t smem = Smem<BN, STAGES>::kBytes;
+    constexpr int kA = (MODE == kUpSwiglu && BN >= 64) ? 2 * kARows : kARows;
+    const size_t smem = Smem<BN, STAGES, kA>::kBytes;
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
     return launch_k(kern, dim3(device_info().sm_count), dim3(kThreads), smem, s, pdl, tA, tB, g);
 }
@@ -517,8 +552,7 @@ cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const int bn = pick_bn(a);
     if (a.act == 0) {
         if (bn == 32) return run<kUpSwiglu, 32, 8>(a, g, a.w1, pdl, s);
-        if (bn == 128) return run<kUpSwiglu, 128, 5>(a, g, a.w1, pdl, s);
-        return run<kUpSwiglu, 256, 4>(a, g, a.w1, pdl, s);
+        return run<kUpSwiglu, 128, 4>(a, g, a.w1, pdl, s);   // two accumulators: 4 x 128 TMEM columns
     }
     if (bn == 32) return run<kUpRelu2, 32, 8>(a, g, a.w1, pdl, s);
     if (bn == 128) return run<kUpRelu2, 128, 5>(a, g, a.w1, pdl, s);
