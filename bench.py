@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="only W + K plain forward calls (for a profiler); prints the work model")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-stages", action="store_true", help="skip the per-stage time breakdown")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-baseline sample")
     return ap.parse_args()
@@ -415,10 +416,41 @@ def main():
                             "peak_source": pk_kind}
     step_s = ms / K / 1e3
     t_hbm = wm["step_bytes"] / (pk["hbm_gbs"] * 1e9)
-    t_tc = wm["flops"] / (pk["bf16_tflops"] * 1e12)
+    t_tc = wm["flops"] / (pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * 1e12)
     line["step_roofline"] = {"bound": "hbm" if t_hbm >= t_tc else "tensor",
                              "roofline_us": max(t_hbm, t_tc) * 1e6, "measured_us": step_s * 1e6,
                              "frac": max(t_hbm, t_tc) / step_s, "bytes": wm["step_bytes"], "flops": wm["flops"]}
+
+    # in-situ time of each stage: graphs of B steps with events around one stage
+    if not args.no_stages:
+        names = [(abi.MOE_STAGE_ROUTE, "route"), (abi.MOE_STAGE_PLAN, "plan"), (abi.MOE_STAGE_UP, "up"),
+                 (abi.MOE_STAGE_DOWN, "down"), (abi.MOE_STAGE_FINAL, "finalize")]
+        stage_us = {}
+        for sid, nm in names:
+            if sid == abi.MOE_STAGE_PLAN and wl.T <= 32:
+                stage_us[nm] = "fused into route"     # one CTA routes and plans at T <= 32
+                continue
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(B_steps)]
+            with torch.cuda.stream(stream):
+                for a_, b_ in evs:
+                    a_.record(stream)
+                    b_.record(stream)
+            stream.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(B_steps):
+                    api.moe_profile_hook(evs[j][0], evs[j][1], sid)
+                    forward(Ws[j % n_sets])
+            api.moe_profile_hook(None, None, 0)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    g.replay()
+            stream.synchronize()
+            vals = [a_.elapsed_time(b_) for a_, b_ in evs]
+            stage_us[nm] = round(1e3 * statistics.mean(vals), 2)
+            del g
+        line["stage_us"] = stage_us
 
     # end to end through the public host-buffer call
     if not args.no_e2e:

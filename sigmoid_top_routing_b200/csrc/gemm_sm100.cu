@@ -45,7 +45,8 @@ using namespace sm100;
 
 constexpr int kBK = 64;                  // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kARows = 128 * kBK * 2;    // 16 KB: 128 weight rows of one k-block
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;            // bf16 weights: producer, MMA, 4 epilogue warps
+constexpr int kThreadsA4 = 320;          // affine 4-bit weights: + 4 dequantisation warps
 
 enum Mode { kUpSwiglu = 0, kUpRelu2 = 1, kDown = 2 };
 
@@ -61,16 +62,19 @@ struct GemmParams {
     int K;                   // reduction length: H (up) or I (down)
     int rows_per_expert;     // rows of the A tensor per expert: 2I, I or H
     int feats;               // output features per expert: I (up) or H (down)
+    const uint16_t* wscale;  // affine 4-bit: (E, rows_per_expert, K/64) bf16 scales
+    const uint16_t* wbias;   //                and biases
     int* err;
 };
 
-template <int BN, int STAGES, int ASTAGE>
+template <int BN, int STAGES, int ASTAGE, int CSTAGE>
 struct Smem {
     static constexpr int kBStage = BN * 128;
     static constexpr size_t kA = 0;
     static constexpr size_t kB = kA + size_t(STAGES) * ASTAGE;
-    static constexpr size_t kBar = kB + size_t(STAGES) * kBStage;           // 8-byte barriers
-    static constexpr int kNumBar = 2 * STAGES + 4 + 1;                      // full, empty, tfull[2], tempty[2], drain
+    static constexpr size_t kC = kB + size_t(STAGES) * kBStage;             // packed 4-bit codes (affine)
+    static constexpr size_t kBar = kC + size_t(STAGES) * CSTAGE;            // 8-byte barriers
+    static constexpr int kNumBar = 3 * STAGES + 4 + 1;   // full, empty, cfull, tfull[2], tempty[2], drain
     static constexpr size_t kMisc = kBar + kNumBar * 8;                       // tmem base, abort flag
     static constexpr size_t kTileBase = kMisc + 16;                           // 257 ints
     static constexpr size_t kTok = kTileBase + 257 * 4;                       // BN ints (token of column)
@@ -120,8 +124,35 @@ MOE_DEV void cp_async_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-template <int MODE, int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+// Dequantise one 128-byte A row (64 affine 4-bit codes of one k-block, one
+// group) into the 128-byte-swizzled bf16 layout: (0x4300 | q) is bf16(128 + q)
+// exactly, minus 128 gives q exactly, and one bf16x2 fma gives
+// bf16_rn(scale * q + bias) with a single rounding.
+MOE_DEV void dequant_row(const uint32_t* codes, uint16_t scale, uint16_t bias, unsigned char* arow, int r) {
+    const uint32_t s2u = uint32_t(scale) | (uint32_t(scale) << 16);
+    const uint32_t b2u = uint32_t(bias) | (uint32_t(bias) << 16);
+    const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+    const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&b2u);
+    const uint32_t k128u = 0x43004300u;
+    const __nv_bfloat162 k128 = *reinterpret_cast<const __nv_bfloat162*>(&k128u);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint32_t w = codes[c];
+        uint32_t o[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const uint32_t t = w >> (8 * p);
+            const uint32_t q2u = (t & 0xFu) | ((t << 12) & 0xF0000u) | 0x43004300u;
+            const __nv_bfloat162 q2 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&q2u), k128);
+            const __nv_bfloat162 v = __hfma2(q2, s2, b2);
+            o[p] = *reinterpret_cast<const uint32_t*>(&v);
+        }
+        *reinterpret_cast<uint4*>(arow + (((c ^ (r & 7)) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+template <int MODE, int BN, int STAGES, int WFMT>
+__global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams g) {
     // SwiGLU with wide token tiles keeps two accumulators (128 gate rows and
     // 128 up rows against one token tile) so a thread holds gate and up of its
@@ -130,7 +161,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool kDual = MODE == kUpSwiglu && BN >= 64;
     constexpr int kAStage = kDual ? 2 * kARows : kARows;
     constexpr int kBoxRows = BN < 64 ? 16 : 64;       // token rows per TMA box
-    using L = Smem<BN, STAGES, kAStage>;
+    // affine 4-bit: the A stage is written by the dequantisation warps from
+    // packed codes (a quarter of the bf16 bytes) staged by TMA
+    constexpr int kCStage = WFMT ? kAStage / 4 : 0;
+    using L = Smem<BN, STAGES, kAStage, kCStage>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sA = sm + L::kA;
@@ -141,6 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = bars + 2 * STAGES;
     uint64_t* tempty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
+    uint64_t* cfull = bars + 2 * STAGES + 5;              // codes landed (affine)
+    unsigned char* sC = sm + L::kC;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
     int* s_base = reinterpret_cast<int*>(sm + L::kTileBase);
@@ -155,12 +191,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // decode-width up tiles gather token rows from x with cp.async (32 lanes + the
     // expect_tx arrive); wider tiles take rows of xs (up) or h (down) by TMA
     constexpr bool kGather = MODE != kDown && BN <= 32;
-    constexpr uint32_t kFullCount = kGather ? 33 : 1;
+    constexpr uint32_t kFullCount = (kGather ? 33 : 1) + (WFMT ? 128 : 0);   // + 128 dequant threads
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], kFullCount);
             mbar_init(&empty[s], 1);
+            if (WFMT) mbar_init(&cfull[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -241,17 +278,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 if (lane == 0) {
                     const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
-                    const uint32_t bytes = kAStage + (kGather ? 0 : nbox * kBoxRows * 128);
+                    const uint32_t bytes = (WFMT ? 0 : kAStage) + (kGather ? 0 : nbox * kBoxRows * 128);
                     mbar_arrive_expect_tx(&full[s], bytes);
-                    unsigned char* a = sA + size_t(s) * kAStage;
+                    if (WFMT) mbar_arrive_expect_tx(&cfull[s], kCStage);
+                    // bf16: weight rows straight into the A stage; affine: codes into the staging area
+                    unsigned char* a = WFMT ? sC + size_t(s) * kCStage : sA + size_t(s) * kAStage;
+                    constexpr int kHalf = WFMT ? kCStage / 2 : kAStage / 2;
+                    const int ax = WFMT ? kb * 8 : kb * kBK;      // codes: 8 words per row per k-block
                     // A: [gate | up] halves for SwiGLU (64 or 128 rows each), else 128 rows
+                    uint64_t* abar = WFMT ? &cfull[s] : &full[s];
                     if (hint_w) {
-                        tma_load_2d_hint(a, &tmA, kb * kBK, a_row, &full[s], pol_w);
-                        if (MODE == kUpSwiglu)
-                            tma_load_2d_hint(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s], pol_w);
+                        tma_load_2d_hint(a, &tmA, ax, a_row, abar, pol_w);
+                        if (MODE == kUpSwiglu) tma_load_2d_hint(a + kHalf, &tmA, ax, a_row + g.I, abar, pol_w);
                     } else {
-                        tma_load_2d(a, &tmA, kb * kBK, a_row, &full[s]);
-                        if (MODE == kUpSwiglu) tma_load_2d(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, &full[s]);
+                        tma_load_2d(a, &tmA, ax, a_row, abar);
+                        if (MODE == kUpSwiglu) tma_load_2d(a + kHalf, &tmA, ax, a_row + g.I, abar);
                     }
                     if (!kGather) {
                         unsigned char* b = sB + size_t(s) * L::kBStage;
@@ -324,6 +365,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(drain, 0, nullptr);
         }
         __syncwarp();
+    } else if (WFMT && warp >= 6) {
+        // ------------------------------------------------------------ dequantisation (affine 4-bit)
+        // Thread dt owns A row dt (and row 128 + dt with two accumulators); its
+        // scale and bias for the next stage are loaded one stage ahead.
+        const int dt = threadIdx.x - 192;
+        constexpr int kRowsPerThread = kDual ? 2 : 1;
+        const int halfr = kDual ? 128 : 64;                // SwiGLU: rows of the gate half
+        const size_t nrows = (size_t)g.E * g.rows_per_expert;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        // global weight row of A row r of tile (e, wt)
+        auto grow = [&](const Tile& tl, int r) -> size_t {
+            const size_t base = (size_t)tl.e * g.rows_per_expert;
+            if (MODE == kUpSwiglu)
+                return r < halfr ? base + (size_t)tl.wt * halfr + r : base + g.I + (size_t)tl.wt * halfr + (r - halfr);
+            return base + (size_t)tl.wt * 128 + r;
+        };
+        auto load_sb = [&](const Tile& tl, int kb, uint16_t (&sc)[2], uint16_t (&bi)[2]) {
+#pragma unroll
+            for (int j = 0; j < kRowsPerThread; ++j) {
+                const size_t gr = grow(tl, dt + 128 * j);
+                if (gr < nrows) {
+                    const size_t gi = gr * g.K / 64 + kb;
+                    sc[j] = __ldg(g.wscale + gi);
+                    bi[j] = __ldg(g.wbias + gi);
+                } else {
+                    sc[j] = 0;
+                    bi[j] = 0;
+                }
+            }
+        };
+        uint16_t nsc[2] = {0, 0}, nbi[2] = {0, 0};
+        int t = blockIdx.x;
+        if (t < total) load_sb(decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets), 0, nsc, nbi);
+        for (; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const int tn = t + gridDim.x;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const uint16_t csc[2] = {nsc[0], nsc[1]}, cbi[2] = {nbi[0], nbi[1]};
+                if (kb + 1 < nkb) load_sb(tl, kb + 1, nsc, nbi);
+                else if (tn < total) load_sb(decode_tile<BN>(tn, s_base, g.E, g.counts, g.offsets), 0, nsc, nbi);
+                if (!mbar_wait(&cfull[s], ph, s_abort)) { ok = false; break; }
+                const uint32_t* cbase = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage);
+                unsigned char* abase = sA + size_t(s) * kAStage;
+#pragma unroll
+                for (int j = 0; j < kRowsPerThread; ++j) {
+                    const int r = dt + 128 * j;           // row of the A stage (rows of 128 bytes)
+                    uint32_t cw[8];
+                    const uint4* cr = reinterpret_cast<const uint4*>(cbase + r * 8);
+                    const uint4 c0 = cr[0], c1 = cr[1];
+                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+                    cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
+                    dequant_row(cw, csc[j], cbi[j], abase + r * 128, r);
+                }
+                fence_proxy_async_smem();                 // generic-proxy writes -> tensor core reads
+                mbar_arrive(&full[s]);
+                if (++s == STAGES) { s = 0; ph ^= 1; }
+            }
+        }
+        if (!ok) {
+            report_error(g.err, kErrWaitExpired);
+            *s_abort = 1;
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         // The four warps run the same tile sequence and the same named
@@ -465,12 +570,31 @@ cudaError_t make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int MODE, int BN, int STAGES>
+// uint32 matrix (outer rows x inner words), no swizzle: packed 4-bit codes.
+cudaError_t make_tmap_u32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                          uint32_t box_outer) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 4};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int MODE, int BN, int STAGES, int WFMT>
 cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, bool pdl, cudaStream_t s) {
     CUtensorMap tA, tB;
     const uint32_t a_box = (MODE == kUpSwiglu && BN < 64) ? 64 : 128;
     const uint32_t b_box = BN < 64 ? 16 : 64;
-    cudaError_t e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E * g.rows_per_expert, kBK, a_box);
+    cudaError_t e;
+    if (WFMT)   // 8 code words (64 codes) of one k-block per row
+        e = make_tmap_u32(&tA, wbase, (uint64_t)g.K / 8, (uint64_t)g.E * g.rows_per_expert, 8, a_box);
+    else
+        e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E * g.rows_per_expert, kBK, a_box);
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
         e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, b_box);
@@ -480,11 +604,14 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
         e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);          // unused (cp.async gather)
     }
     if (e != cudaSuccess) return e;
-    auto kern = k_gemm<MODE, BN, STAGES>;
+    auto kern = k_gemm<MODE, BN, STAGES, WFMT>;
     constexpr int kA = (MODE == kUpSwiglu && BN >= 64) ? 2 * kARows : kARows;
-    const size_t smem = Smem<BN, STAGES, kA>::kBytes;
+    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0>;
+    static_assert(L::kBytes <= 227 * 1024, "shared memory of one CTA");
+    const size_t smem = L::kBytes;
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
-    return launch_k(kern, dim3(device_info().sm_count), dim3(kThreads), smem, s, pdl, tA, tB, g);
+    return launch_k(kern, dim3(device_info().sm_count), dim3(WFMT ? kThreadsA4 : kThreads), smem, s, pdl, tA,
+                    tB, g);
 }
 
 // Token-tile width from the mean pairs per expert.
@@ -513,10 +640,14 @@ GemmParams params(const ExpertArgs& a, bool up) {
         g.K = a.H;
         g.rows_per_expert = a.act == 0 ? 2 * a.I : a.I;
         g.feats = a.I;
+        g.wscale = a.w1_scale;
+        g.wbias = a.w1_bias;
     } else {
         g.K = a.I;
         g.rows_per_expert = a.H;
         g.feats = a.H;
+        g.wscale = a.w2_scale;
+        g.wbias = a.w2_bias;
     }
     return g;
 }
@@ -537,7 +668,7 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict_
 
 }  // namespace
 
-bool gemm_needs_xs(const ExpertArgs& a) { return a.fmt == 0 && pick_bn(a) > 32; }
+bool gemm_needs_xs(const ExpertArgs& a) { return pick_bn(a) > 32; }
 
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const int P = a.T * a.k;
@@ -547,25 +678,37 @@ cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
 }
 
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    if (a.fmt != 0) return cudaErrorNotSupported;
     const GemmParams g = params(a, true);
     const int bn = pick_bn(a);
-    if (a.act == 0) {
-        if (bn == 32) return run<kUpSwiglu, 32, 8>(a, g, a.w1, pdl, s);
-        return run<kUpSwiglu, 128, 4>(a, g, a.w1, pdl, s);   // two accumulators: 4 x 128 TMEM columns
+    if (a.fmt == 0) {
+        if (a.act == 0) {
+            if (bn == 32) return run<kUpSwiglu, 32, 8, 0>(a, g, a.w1, pdl, s);
+            return run<kUpSwiglu, 128, 4, 0>(a, g, a.w1, pdl, s);   // two accumulators: 4 x 128 TMEM columns
+        }
+        if (bn == 32) return run<kUpRelu2, 32, 8, 0>(a, g, a.w1, pdl, s);
+        if (bn == 128) return run<kUpRelu2, 128, 5, 0>(a, g, a.w1, pdl, s);
+        return run<kUpRelu2, 256, 4, 0>(a, g, a.w1, pdl, s);
     }
-    if (bn == 32) return run<kUpRelu2, 32, 8>(a, g, a.w1, pdl, s);
-    if (bn == 128) return run<kUpRelu2, 128, 5>(a, g, a.w1, pdl, s);
-    return run<kUpRelu2, 256, 4>(a, g, a.w1, pdl, s);
+    if (a.act == 0) {
+        if (bn == 32) return run<kUpSwiglu, 32, 8, 1>(a, g, a.w1, pdl, s);
+        return run<kUpSwiglu, 128, 3, 1>(a, g, a.w1, pdl, s);
+    }
+    if (bn == 32) return run<kUpRelu2, 32, 8, 1>(a, g, a.w1, pdl, s);
+    if (bn == 128) return run<kUpRelu2, 128, 5, 1>(a, g, a.w1, pdl, s);
+    return run<kUpRelu2, 256, 4, 1>(a, g, a.w1, pdl, s);
 }
 
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    if (a.fmt != 0) return cudaErrorNotSupported;
     const GemmParams g = params(a, false);
     const int bn = pick_bn(a);
-    if (bn == 32) return run<kDown, 32, 8>(a, g, a.w2, pdl, s);
-    if (bn == 128) return run<kDown, 128, 5>(a, g, a.w2, pdl, s);
-    return run<kDown, 256, 4>(a, g, a.w2, pdl, s);
+    if (a.fmt == 0) {
+        if (bn == 32) return run<kDown, 32, 8, 0>(a, g, a.w2, pdl, s);
+        if (bn == 128) return run<kDown, 128, 5, 0>(a, g, a.w2, pdl, s);
+        return run<kDown, 256, 4, 0>(a, g, a.w2, pdl, s);
+    }
+    if (bn == 32) return run<kDown, 32, 8, 1>(a, g, a.w2, pdl, s);
+    if (bn == 128) return run<kDown, 128, 5, 1>(a, g, a.w2, pdl, s);
+    return run<kDown, 256, 4, 1>(a, g, a.w2, pdl, s);
 }
 
 }  // namespace moe

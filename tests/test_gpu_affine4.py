@@ -1,0 +1,65 @@
+"""Parity of the MLX-style affine 4-bit expert path (codes dequantised on chip
+into the tcgen05 operand) with the float64 oracle, which dequantises the same
+codes exactly.  Gate: rel-L2 <= 3e-2 (the weights are rounded once to bf16
+on chip, the oracle keeps them exact)."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from sigmoid_top_routing_b200 import inputs as G
+from tests.test_gpu_parity import _check_all, inputs_of, run_forward
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def api():
+    from sigmoid_top_routing_b200 import build
+    build.build(quiet=True)
+    from sigmoid_top_routing_b200 import api as A
+    A.load()
+    return A
+
+
+def test_affine4_small_ragged(api):
+    """Decode-width tiles (token tiles of 32), I = 64 (one SwiGLU tile), E = 8."""
+    wl = G.Workload("a4_small", T=33, H=128, E=8, k=4, I=64, fmt="affine4")
+    inp = inputs_of(wl)
+    _check_all(inp, run_forward(api, inp))
+
+
+def test_affine4_relu2_small(api):
+    wl = G.Workload("a4_relu2", T=40, H=256, E=16, k=6, I=192, act="relu2", fmt="affine4", out_scale=2.5)
+    inp = inputs_of(wl)
+    _check_all(inp, run_forward(api, inp))
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_affine4_decode_sizes(api, T):
+    inp = inputs_of(G.WORKLOADS[f"affine4_t{T}"])
+    _check_all(inp, run_forward(api, inp))
+
+
+def test_affine4_t512(api):
+    """Token tiles of 128: two accumulators (gate, up) per SwiGLU tile."""
+    inp = inputs_of(G.WORKLOADS["affine4_t512"])
+    _check_all(inp, run_forward(api, inp))
+
+
+def test_affine4_t8192_sampled(api):
+    """The full 8192-token workload as the benchmark runs it; 384 sampled
+    rows against the oracle, plus the whole plan."""
+    inp = inputs_of(G.WORKLOADS["affine4_t8192"])
+    out = run_forward(api, inp)
+    tokens = np.sort(np.random.default_rng(7).choice(inp.wl.T, 384, replace=False))
+    _check_all(inp, out, tokens=tokens)
+
+
+def test_affine4_relu2_wide_tiles(api):
+    """relu^2 with token tiles of 256 (mean pairs per expert > 96)."""
+    wl = G.Workload("a4_relu2_wide", T=1024, H=256, E=8, k=2, I=320, act="relu2", fmt="affine4")
+    inp = inputs_of(wl)
+    _check_all(inp, run_forward(api, inp))
