@@ -46,7 +46,8 @@ using namespace sm100;
 constexpr int kBK = 64;                  // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kARows = 128 * kBK * 2;    // 16 KB: 128 weight rows of one k-block
 constexpr int kThreads = 192;            // bf16 weights: producer, MMA, 4 epilogue warps
-constexpr int kThreadsA4 = 320;          // affine 4-bit weights: + 4 dequantisation warps
+constexpr int kThreadsA4 = 448;          // affine 4-bit weights: + 8 dequantisation warps
+constexpr int kSBDepth = 4;              // stages of scales/biases in flight per dequant thread
 
 enum Mode { kUpSwiglu = 0, kUpRelu2 = 1, kDown = 2 };
 
@@ -67,7 +68,7 @@ struct GemmParams {
     int* err;
 };
 
-template <int BN, int STAGES, int ASTAGE, int CSTAGE>
+template <int BN, int STAGES, int ASTAGE, int CSTAGE, int SBRING = (CSTAGE ? kSBDepth * 2 * 256 * 4 : 0)>
 struct Smem {
     static constexpr int kBStage = BN * 128;
     static constexpr size_t kA = 0;
@@ -81,7 +82,8 @@ struct Smem {
     static constexpr size_t kTokW = kTok + BN * 4;                            // BN floats
     static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats
     static constexpr size_t kTrow = kU + 64 * 17 * 4;                         // BN ints (producer's token rows)
-    static constexpr size_t kEnd = kTrow + BN * 4;
+    static constexpr size_t kSB = kTrow + BN * 4;                             // scale/bias ring (affine)
+    static constexpr size_t kEnd = kSB + SBRING;
     static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
 };
 
@@ -124,11 +126,15 @@ MOE_DEV void cp_async_arrive(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Dequantise one 128-byte A row (64 affine 4-bit codes of one k-block, one
-// group) into the 128-byte-swizzled bf16 layout: (0x4300 | q) is bf16(128 + q)
-// exactly, minus 128 gives q exactly, and one bf16x2 fma gives
+// Dequantise 16-byte chunks [c0, c0 + NC) of one 128-byte A row (8 affine
+// 4-bit codes per chunk, one group per row per k-block) into the 128-byte-
+// swizzled bf16 layout.  The low and high nibbles of a code word are split
+// into byte lanes, PRMT pairs codes (2p, 2p + 1) and OR 0x4300 makes
+// bf16(128 + q) exactly; minus 128 gives q exactly and one bf16x2 fma gives
 // bf16_rn(scale * q + bias) with a single rounding.
-MOE_DEV void dequant_row(const uint32_t* codes, uint16_t scale, uint16_t bias, unsigned char* arow, int r) {
+template <int NC>
+MOE_DEV void dequant_chunks(const uint32_t* codes, int c0, uint16_t scale, uint16_t bias, unsigned char* arow,
+                            int r) {
     const uint32_t s2u = uint32_t(scale) | (uint32_t(scale) << 16);
     const uint32_t b2u = uint32_t(bias) | (uint32_t(bias) << 16);
     const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
@@ -136,13 +142,18 @@ MOE_DEV void dequant_row(const uint32_t* codes, uint16_t scale, uint16_t bias, u
     const uint32_t k128u = 0x43004300u;
     const __nv_bfloat162 k128 = *reinterpret_cast<const __nv_bfloat162*>(&k128u);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint32_t w = codes[c];
+    for (int i = 0; i < NC; ++i) {
+        const int c = c0 + i;
+        const uint32_t w = codes[i];
+        const uint32_t lo = w & 0x0F0F0F0Fu;           // codes 0, 2, 4, 6 in bytes 0..3
+        const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;    // codes 1, 3, 5, 7
         uint32_t o[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            const uint32_t t = w >> (8 * p);
-            const uint32_t q2u = (t & 0xFu) | ((t << 12) & 0xF0000u) | 0x43004300u;
+            const uint32_t sel = uint32_t(p) | (uint32_t(p) << 4) | (uint32_t(4 + p) << 8) | (uint32_t(4 + p) << 12);
+            uint32_t x;
+            asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(lo), "r"(hi), "r"(sel));
+            const uint32_t q2u = (x & 0x00FF00FFu) | 0x43004300u;
             const __nv_bfloat162 q2 = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&q2u), k128);
             const __nv_bfloat162 v = __hfma2(q2, s2, b2);
             o[p] = *reinterpret_cast<const uint32_t*>(&v);
@@ -150,6 +161,13 @@ MOE_DEV void dequant_row(const uint32_t* codes, uint16_t scale, uint16_t bias, u
         *reinterpret_cast<uint4*>(arow + (((c ^ (r & 7)) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
+
+MOE_DEV void cp_async4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+MOE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int MODE, int BN, int STAGES, int WFMT>
 __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
@@ -191,7 +209,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     // decode-width up tiles gather token rows from x with cp.async (32 lanes + the
     // expect_tx arrive); wider tiles take rows of xs (up) or h (down) by TMA
     constexpr bool kGather = MODE != kDown && BN <= 32;
-    constexpr uint32_t kFullCount = (kGather ? 33 : 1) + (WFMT ? 128 : 0);   // + 128 dequant threads
+    constexpr uint32_t kFullCount = (kGather ? 33 : 1) + (WFMT ? 256 : 0);   // + 256 dequant threads
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -365,66 +383,80 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             mbar_wait(drain, 0, nullptr);
         }
         __syncwarp();
-    } else if (WFMT && warp >= 6) {
+    } else if (WFMT && warp >= 6) {   // warps 6..13
         // ------------------------------------------------------------ dequantisation (affine 4-bit)
-        // Thread dt owns A row dt (and row 128 + dt with two accumulators); its
-        // scale and bias for the next stage are loaded one stage ahead.
+        // 256 threads.  Thread dt owns A row r (two threads per row at decode
+        // width, each half of its 8 chunks).  Each thread fetches its row's
+        // scale and bias kSBDepth stages ahead with 4-byte cp.async into a ring
+        // in shared memory (the word holding the bf16; the half is picked later).
         const int dt = threadIdx.x - 192;
-        constexpr int kRowsPerThread = kDual ? 2 : 1;
+        constexpr int kCPT = kDual ? 8 : 4;
+        const int r = kDual ? dt : (dt >> 1);
+        const int cbeg = kDual ? 0 : (dt & 1) * 4;
         const int halfr = kDual ? 128 : 64;                // SwiGLU: rows of the gate half
         const size_t nrows = (size_t)g.E * g.rows_per_expert;
-        int s = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        // global weight row of A row r of tile (e, wt)
-        auto grow = [&](const Tile& tl, int r) -> size_t {
+        const int G = g.K / 64;
+        uint32_t* s_sb = reinterpret_cast<uint32_t*>(sm + L::kSB);
+        auto grow = [&](const Tile& tl) -> size_t {      // global weight row of A row r
             const size_t base = (size_t)tl.e * g.rows_per_expert;
             if (MODE == kUpSwiglu)
                 return r < halfr ? base + (size_t)tl.wt * halfr + r : base + g.I + (size_t)tl.wt * halfr + (r - halfr);
             return base + (size_t)tl.wt * 128 + r;
         };
-        auto load_sb = [&](const Tile& tl, int kb, uint16_t (&sc)[2], uint16_t (&bi)[2]) {
-#pragma unroll
-            for (int j = 0; j < kRowsPerThread; ++j) {
-                const size_t gr = grow(tl, dt + 128 * j);
-                if (gr < nrows) {
-                    const size_t gi = gr * g.K / 64 + kb;
-                    sc[j] = __ldg(g.wscale + gi);
-                    bi[j] = __ldg(g.wbias + gi);
-                } else {
-                    sc[j] = 0;
-                    bi[j] = 0;
+        // look-ahead iterator over this CTA's (tile, k-block) stages
+        int at = blockIdx.x, akb = 0;
+        Tile atl{};
+        if (at < total) atl = decode_tile<BN>(at, s_base, g.E, g.counts, g.offsets);
+        auto issue = [&](int slot) {
+            if (at < total) {
+                const size_t gr = grow(atl);
+                const size_t gi = gr < nrows ? gr * G + akb : 0;
+                cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt), g.wscale + (gi & ~size_t(1)));
+                cp_async4(smem_u32(s_sb + (slot * 2 + 1) * 256 + dt), g.wbias + (gi & ~size_t(1)));
+                if (++akb == nkb) {
+                    akb = 0;
+                    at += gridDim.x;
+                    if (at < total) atl = decode_tile<BN>(at, s_base, g.E, g.counts, g.offsets);
                 }
             }
+            cp_async_commit();
         };
-        uint16_t nsc[2] = {0, 0}, nbi[2] = {0, 0};
-        int t = blockIdx.x;
-        if (t < total) load_sb(decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets), 0, nsc, nbi);
-        for (; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
-            const int tn = t + gridDim.x;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const uint16_t csc[2] = {nsc[0], nsc[1]}, cbi[2] = {nbi[0], nbi[1]};
-                if (kb + 1 < nkb) load_sb(tl, kb + 1, nsc, nbi);
-                else if (tn < total) load_sb(decode_tile<BN>(tn, s_base, g.E, g.counts, g.offsets), 0, nsc, nbi);
-                if (!mbar_wait(&cfull[s], ph, s_abort)) { ok = false; break; }
-                const uint32_t* cbase = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage);
-                unsigned char* abase = sA + size_t(s) * kAStage;
 #pragma unroll
-                for (int j = 0; j < kRowsPerThread; ++j) {
-                    const int r = dt + 128 * j;           // row of the A stage (rows of 128 bytes)
-                    uint32_t cw[8];
-                    const uint4* cr = reinterpret_cast<const uint4*>(cbase + r * 8);
-                    const uint4 c0 = cr[0], c1 = cr[1];
-                    cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
-                    cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
-                    dequant_row(cw, csc[j], cbi[j], abase + r * 128, r);
+        for (int j = 0; j < kSBDepth; ++j) issue(j);
+        int s = 0, slot = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const size_t gr = grow(tl);
+            for (int kb = 0; kb < nkb; ++kb) {
+                cp_async_wait<kSBDepth - 1>();               // this stage's scale/bias landed
+                const uint32_t sw = s_sb[(slot * 2 + 0) * 256 + dt];
+                const uint32_t bw = s_sb[(slot * 2 + 1) * 256 + dt];
+                const bool odd = ((gr * G + kb) & 1) != 0;
+                const bool inb = gr < nrows;
+                const uint16_t sc = inb ? uint16_t(odd ? sw >> 16 : sw & 0xFFFFu) : uint16_t(0);
+                const uint16_t bi = inb ? uint16_t(odd ? bw >> 16 : bw & 0xFFFFu) : uint16_t(0);
+                issue(slot);                                  // refill the slot kSBDepth stages ahead
+                if (++slot == kSBDepth) slot = 0;
+                if (!mbar_wait(&cfull[s], ph, s_abort)) { ok = false; break; }
+                const uint32_t* crow = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage) + r * 8 + cbeg;
+                uint32_t cw[kCPT];
+#pragma unroll
+                for (int q = 0; q < kCPT / 4; ++q) {
+                    const uint4 c4 = reinterpret_cast<const uint4*>(crow)[q];
+                    cw[4 * q + 0] = c4.x;
+                    cw[4 * q + 1] = c4.y;
+                    cw[4 * q + 2] = c4.z;
+                    cw[4 * q + 3] = c4.w;
                 }
+                dequant_chunks<kCPT>(cw, cbeg, sc, bi, sA + size_t(s) * kAStage + r * 128, r);
                 fence_proxy_async_smem();                 // generic-proxy writes -> tensor core reads
                 mbar_arrive(&full[s]);
                 if (++s == STAGES) { s = 0; ph ^= 1; }
             }
         }
+        cp_async_wait<0>();                               // no copy of this thread left in flight
         if (!ok) {
             report_error(g.err, kErrWaitExpired);
             *s_abort = 1;
@@ -606,7 +638,7 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     if (e != cudaSuccess) return e;
     auto kern = k_gemm<MODE, BN, STAGES, WFMT>;
     constexpr int kA = (MODE == kUpSwiglu && BN >= 64) ? 2 * kARows : kARows;
-    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0>;
+    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0>;   // + the scale/bias ring for affine
     static_assert(L::kBytes <= 227 * 1024, "shared memory of one CTA");
     const size_t smem = L::kBytes;
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;

@@ -14,6 +14,7 @@ struct RouteArgs {
     const float* w_router;   // (E, H) fp32
     const float* bias;       // (E) fp32 or null
     float* l_scratch;        // (T, E) fp32 scratch for the small-T logits pass
+    float* part;             // (8, T, E) fp32 per-segment partial logits, or null
     int T, H, E, k;
     float eps, scale;
     int32_t* idx;            // (T, k)

@@ -94,8 +94,10 @@ void layout(const moe_dims* d, moe_ws_layout* L) {
     off = align256(off + P * I * 2);
     L->xs = off;          // token rows gathered in plan order (wide token tiles)
     off = align256(off + P * H * 2);
-    L->scratch = off;     // router logits (T <= 32) | multi-CTA plan histograms and bases
+    // scratch: router logits (T <= 32) | plan histograms and bases | per-segment partial logits
+    L->scratch = off;
     off = align256(off + (size_t)kSmallT * E * 4 + 4096 + plan_scratch_ints((int)P, (int)E) * 4);
+    off = align256(off + (size_t)8 * T * E * 4);
     L->total = off;
 }
 
@@ -105,6 +107,7 @@ struct WsView {
     uint16_t* xs;
     float* l_scratch;
     int32_t* plan_scratch;
+    float* part;
 };
 
 moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
@@ -119,7 +122,10 @@ moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
     v->h = reinterpret_cast<uint16_t*>(b + L.h);
     v->xs = reinterpret_cast<uint16_t*>(b + L.xs);
     v->l_scratch = reinterpret_cast<float*>(b + L.scratch);
-    v->plan_scratch = reinterpret_cast<int32_t*>(b + L.scratch + (size_t)kSmallT * d->E * 4 + 4096);
+    const size_t off_plan = L.scratch + (size_t)kSmallT * d->E * 4 + 4096;
+    v->plan_scratch = reinterpret_cast<int32_t*>(b + off_plan);
+    v->part = reinterpret_cast<float*>(
+        b + align256(off_plan + plan_scratch_ints(d->T * d->k, d->E) * 4));
     return MOE_OK;
 }
 
@@ -390,6 +396,7 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
     r.w_router = w_router;
     r.bias = expert_bias;
     r.l_scratch = v.l_scratch;
+    r.part = v.part;
     r.T = d->T;
     r.H = d->H;
     r.E = d->E;

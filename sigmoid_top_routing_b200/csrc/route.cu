@@ -101,8 +101,10 @@ MOE_DEV void zero_slice(const RouteArgs& a) {
     if (!a.zero_ptr) return;
     const size_t n4 = a.zero_count / 4;
     float4* p = reinterpret_cast<float4*>(a.zero_ptr);
-    const size_t stride = (size_t)gridDim.x * blockDim.x;
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
+    const size_t blocks = (size_t)gridDim.x * gridDim.y;
+    const size_t block = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    const size_t stride = blocks * blockDim.x;
+    for (size_t i = block * blockDim.x + threadIdx.x; i < n4; i += stride)
         p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(256) k_logits_small(RouteArgs a) {
 // ---------------------------------------------------------------------------
 // Selection from fp32 logits in memory; FUSE also builds the plan (one CTA,
 // T <= 32 so P <= 1024).
-template <int NE, bool FUSE>
+template <int NE, bool FUSE, bool PART>
 __global__ void __launch_bounds__(256) k_select(RouteArgs a) {
     __shared__ int s_idx[FUSE ? 1024 : 1];
     __shared__ int s_cnt[FUSE ? 256 : 1], s_off[FUSE ? 257 : 1], s_til[FUSE ? 257 : 1];
@@ -167,7 +169,17 @@ __global__ void __launch_bounds__(256) k_select(RouteArgs a) {
 #pragma unroll
         for (int i = 0; i < NE; ++i) {
             const int e = lane + 32 * i;
-            Lv[i] = e < a.E ? L[(size_t)t * a.E + e] : 0.0f;
+            if (PART) {       // L = p_0 + p_1 + ... + p_7, left to right
+                float L = 0.0f;
+                if (e < a.E) {
+                    L = a.part[(size_t)t * a.E + e];
+#pragma unroll
+                    for (int w = 1; w < kSegs; ++w) L += a.part[((size_t)w * a.T + t) * a.E + e];
+                }
+                Lv[i] = L;
+            } else {
+                Lv[i] = e < a.E ? L[(size_t)t * a.E + e] : 0.0f;
+            }
         }
         const int e = select_token<NE>(Lv, a.bias, a.E, a.k, a.eps, a.scale, a.idx + (size_t)t * a.k,
                                        a.w + (size_t)t * a.k);
@@ -350,17 +362,182 @@ cudaError_t run_large(const RouteArgs& a, bool pdl, cudaStream_t s) {
     return launch_k(kern, dim3((a.T + TT - 1) / TT), dim3(256), smem, s, pdl, a);
 }
 
-template <int NE>
+template <int NE, bool PART>
 cudaError_t run_select(const RouteArgs& a, bool fuse, bool pdl, cudaStream_t s) {
-    if (fuse) return launch_k(k_select<NE, true>, dim3(1), dim3(256), 0, s, pdl, a);
-    return launch_k(k_select<NE, false>, dim3((a.T + 7) / 8), dim3(256), 0, s, pdl, a);
+    if (fuse) return launch_k(k_select<NE, true, PART>, dim3(1), dim3(256), 0, s, pdl, a);
+    return launch_k(k_select<NE, false, PART>, dim3((a.T + 7) / 8), dim3(256), 0, s, pdl, a);
 }
 
+template <bool PART>
 cudaError_t dispatch_select(const RouteArgs& a, bool fuse, bool pdl, cudaStream_t s) {
-    if (a.E <= 32) return run_select<1>(a, fuse, pdl, s);
-    if (a.E <= 64) return run_select<2>(a, fuse, pdl, s);
-    if (a.E <= 128) return run_select<4>(a, fuse, pdl, s);
-    return run_select<8>(a, fuse, pdl, s);
+    if (a.E <= 32) return run_select<1, PART>(a, fuse, pdl, s);
+    if (a.E <= 64) return run_select<2, PART>(a, fuse, pdl, s);
+    if (a.E <= 128) return run_select<4, PART>(a, fuse, pdl, s);
+    return run_select<8, PART>(a, fuse, pdl, s);
+}
+
+// ---------------------------------------------------------------------------
+// Segment partials: each CTA computes one segment's fmaf chains (the
+// canonical order above) for a block of tokens and all experts and writes
+// p_w[t][e]; k_select<.., PART> then forms L = p_0 + ... + p_7 in order, so
+// these logits are bit-identical to the one-CTA kernels', with 8x the CTAs.
+
+// T <= 32: CTA (expert e, segment w), one warp, lane = token; the next
+// chunk's token values and router row are loaded while this one is summed.
+__global__ void __launch_bounds__(32) k_logits_seg_small(RouteArgs a) {
+    pdl_wait();
+    zero_slice(a);
+    const int e = blockIdx.x, w = blockIdx.y, lane = threadIdx.x;
+    const int H = a.H;
+    const int nch = (H / kChunk - w + kSegs - 1) / kSegs;
+    const bool tv = lane < a.T;
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(tv ? lane : 0) * H);
+    const float4* wr = reinterpret_cast<const float4*>(a.w_router + (size_t)e * H);
+    uint4 xv[4], xn[4];
+    float4 wv[8], wn[8];
+    auto load = [&](int j, uint4 (&xo)[4], float4 (&wo)[8]) {
+        const int h0 = (w + kSegs * j) * kChunk;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xo[q] = ld_nc(xr + h0 / 8 + q);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) wo[q] = __ldg(wr + h0 / 4 + q);
+    };
+    float acc = 0.0f;
+    if (nch > 0) load(0, xv, wv);
+    for (int j = 0; j < nch; ++j) {
+        if (j + 1 < nch) load(j + 1, xn, wn);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 w0 = wv[2 * q], w1 = wv[2 * q + 1];
+            acc = fmaf(bf16lo(xv[q].x), w0.x, acc);
+            acc = fmaf(bf16hi(xv[q].x), w0.y, acc);
+            acc = fmaf(bf16lo(xv[q].y), w0.z, acc);
+            acc = fmaf(bf16hi(xv[q].y), w0.w, acc);
+            acc = fmaf(bf16lo(xv[q].z), w1.x, acc);
+            acc = fmaf(bf16hi(xv[q].z), w1.y, acc);
+            acc = fmaf(bf16lo(xv[q].w), w1.z, acc);
+            acc = fmaf(bf16hi(xv[q].w), w1.w, acc);
+        }
+        if (j + 1 < nch) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) xv[q] = xn[q];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) wv[q] = wn[q];
+        }
+    }
+    if (tv) a.part[((size_t)w * a.T + lane) * a.E + e] = acc;
+    pdl_trigger();
+}
+
+// Large T: CTA (token block, segment w), 64 threads; thread (tg, eg) owns
+// TPT tokens x EPT experts of the TT x EP block (register-blocked FMAs, the
+// router chunk staged transposed, the token chunk staged as fp32).
+template <int NE, int TT, int TPT, int EPT>
+__global__ void __launch_bounds__(64) k_logits_seg(RouteArgs a) {
+    constexpr int EP = 32 * NE;
+    static_assert(TT == 8 * TPT && EP == 8 * EPT, "thread tiling");
+    constexpr int WF4 = EP * 8 / 64;      // float4 of router values per thread per chunk
+    constexpr int XV4 = TT * 4 / 64;      // uint4 of token values per thread per chunk
+    constexpr bool PF = NE <= 4;          // register prefetch of the next chunk
+    __shared__ __align__(16) float wt[kChunk * EP];
+    __shared__ __align__(16) float xs[kChunk * TT];
+    pdl_wait();
+    zero_slice(a);
+    const int w = blockIdx.y, t0 = blockIdx.x * TT, tid = threadIdx.x;
+    const int tg = tid & 7, eg = tid >> 3;
+    const int E = a.E, H = a.H;
+    const int nch = (H / kChunk - w + kSegs - 1) / kSegs;
+    float acc[TPT][EPT];
+#pragma unroll
+    for (int i = 0; i < TPT; ++i)
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) acc[i][j] = 0.0f;
+    float4 rw[WF4];
+    uint4 rx[XV4 > 0 ? XV4 : 1];
+    auto load = [&](int j) {
+        const int h0 = (w + kSegs * j) * kChunk;
+#pragma unroll
+        for (int i = 0; i < WF4; ++i) {
+            const int f = tid + 64 * i;
+            const int e = f % EP, v = f / EP;              // consecutive threads: consecutive experts
+            rw[i] = e < E ? __ldg(reinterpret_cast<const float4*>(a.w_router + (size_t)e * H + h0) + v)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < XV4; ++i) {
+            const int f = tid + 64 * i;
+            const int t = f % TT, v = f / TT;
+            const bool ok = t0 + t < a.T;
+            rx[i] = ok ? ld_nc(reinterpret_cast<const uint4*>(a.x + (size_t)(t0 + t) * H + h0) + v)
+                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    auto stage = [&]() {
+#pragma unroll
+        for (int i = 0; i < WF4; ++i) {
+            const int f = tid + 64 * i;
+            const int e = f % EP, v = f / EP;
+            wt[(4 * v + 0) * EP + e] = rw[i].x;
+            wt[(4 * v + 1) * EP + e] = rw[i].y;
+            wt[(4 * v + 2) * EP + e] = rw[i].z;
+            wt[(4 * v + 3) * EP + e] = rw[i].w;
+        }
+#pragma unroll
+        for (int i = 0; i < XV4; ++i) {
+            const int f = tid + 64 * i;
+            const int t = f % TT, v = f / TT;
+            xs[(8 * v + 0) * TT + t] = bf16lo(rx[i].x);
+            xs[(8 * v + 1) * TT + t] = bf16hi(rx[i].x);
+            xs[(8 * v + 2) * TT + t] = bf16lo(rx[i].y);
+            xs[(8 * v + 3) * TT + t] = bf16hi(rx[i].y);
+            xs[(8 * v + 4) * TT + t] = bf16lo(rx[i].z);
+            xs[(8 * v + 5) * TT + t] = bf16hi(rx[i].z);
+            xs[(8 * v + 6) * TT + t] = bf16lo(rx[i].w);
+            xs[(8 * v + 7) * TT + t] = bf16hi(rx[i].w);
+        }
+    };
+    if (PF && nch > 0) load(0);
+    for (int j = 0; j < nch; ++j) {
+        if (!PF) load(j);
+        __syncthreads();            // the previous chunk's compute is done with the buffers
+        stage();
+        __syncthreads();
+        if (PF && j + 1 < nch) load(j + 1);
+#pragma unroll 4
+        for (int hh = 0; hh < kChunk; ++hh) {
+            float xv[TPT];
+            if (TPT == 4) {
+                const float4 t4 = *reinterpret_cast<const float4*>(xs + hh * TT + tg * TPT);
+                xv[0] = t4.x; xv[TPT > 1 ? 1 : 0] = t4.y; xv[TPT > 2 ? 2 : 0] = t4.z; xv[TPT > 3 ? 3 : 0] = t4.w;
+            } else {
+                const float2 t2 = *reinterpret_cast<const float2*>(xs + hh * TT + tg * TPT);
+                xv[0] = t2.x; xv[TPT > 1 ? 1 : 0] = t2.y;
+            }
+            const float4* wp = reinterpret_cast<const float4*>(wt + hh * EP + eg * EPT);
+#pragma unroll
+            for (int q = 0; q < EPT / 4; ++q) {
+                const float4 w4 = wp[q];
+#pragma unroll
+                for (int i = 0; i < TPT; ++i) {
+                    acc[i][4 * q + 0] = fmaf(xv[i], w4.x, acc[i][4 * q + 0]);
+                    acc[i][4 * q + 1] = fmaf(xv[i], w4.y, acc[i][4 * q + 1]);
+                    acc[i][4 * q + 2] = fmaf(xv[i], w4.z, acc[i][4 * q + 2]);
+                    acc[i][4 * q + 3] = fmaf(xv[i], w4.w, acc[i][4 * q + 3]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+        const int t = t0 + tg * TPT + i;
+        if (t >= a.T) continue;
+#pragma unroll
+        for (int j = 0; j < EPT; ++j) {
+            const int e = eg * EPT + j;
+            if (e < E) a.part[((size_t)w * a.T + t) * E + e] = acc[i][j];
+        }
+    }
+    pdl_trigger();
 }
 
 }  // namespace
@@ -370,7 +547,27 @@ cudaError_t launch_route(const RouteArgs& a, bool fuse_plan, bool pdl, cudaStrea
     if (a.T == 0) return cudaSuccess;
     *n_launched = 1;
     const bool small = a.T <= kSmallT;
-    if (a.logits) return dispatch_select(a, fuse_plan && small, pdl, s);
+    if (a.logits) return dispatch_select<false>(a, fuse_plan && small, pdl, s);
+    if (a.part) {
+        // per-segment partials (8x the CTAs), then select from their ordered sum
+        cudaError_t e;
+        if (small) {
+            e = launch_k(k_logits_seg_small, dim3(a.E, kSegs), dim3(32), 0, s, pdl, a);
+        } else if (a.E <= 32) {
+            e = launch_k(k_logits_seg<1, 32, 4, 4>, dim3((a.T + 31) / 32, kSegs), dim3(64), 0, s, pdl, a);
+        } else if (a.E <= 64) {
+            e = launch_k(k_logits_seg<2, 32, 4, 8>, dim3((a.T + 31) / 32, kSegs), dim3(64), 0, s, pdl, a);
+        } else if (a.E <= 128) {
+            e = launch_k(k_logits_seg<4, 32, 4, 16>, dim3((a.T + 31) / 32, kSegs), dim3(64), 0, s, pdl, a);
+        } else {
+            e = launch_k(k_logits_seg<8, 16, 2, 32>, dim3((a.T + 15) / 16, kSegs), dim3(64), 0, s, pdl, a);
+        }
+        if (e != cudaSuccess) return e;
+        *n_launched = 2;
+        RouteArgs b = a;
+        b.zero_ptr = nullptr;
+        return dispatch_select<true>(b, fuse_plan && small, pdl, s);
+    }
     if (small && a.l_scratch) {
         // two launches: per-expert logits into scratch (this one also zeroes
         // the accumulator), then select (+ plan)
@@ -382,7 +579,7 @@ cudaError_t launch_route(const RouteArgs& a, bool fuse_plan, bool pdl, cudaStrea
         *n_launched = 2;
         RouteArgs b = a;
         b.zero_ptr = nullptr;
-        return dispatch_select(b, fuse_plan, pdl, s);
+        return dispatch_select<false>(b, fuse_plan, pdl, s);
     }
     if (a.E <= 32) return run_large<1, 32, 32>(a, pdl, s);
     if (a.E <= 64) return run_large<2, 32, 32>(a, pdl, s);

@@ -201,3 +201,28 @@ def test_empty_batch_is_a_no_op(api):
     y = torch.empty((0, wl.H), dtype=torch.bfloat16, device="cuda")
     api.moe_forward(x, D.W, D.w_router, D.expert_bias, E=wl.E, k=wl.k, I=wl.I, y=y)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("base,T", [("lfm2_decode_t8", 8), ("lfm2_prefill_t4096", 4096),
+                                    ("nemotron_relu2_t2048", 2048), ("nemotron_relu2_t2048", 19)])
+def test_forward_router_matches_standalone_router_bitwise(api, base, T):
+    """moe_forward routes through per-segment partial logits (8x the CTAs);
+    moe_route uses one CTA per token block.  Both follow the same fp32 order,
+    so picks and weights must be the same bits."""
+    wl = dataclasses.replace(G.WORKLOADS[base].with_T(T), nan_rows=0)
+    inp = G.make_inputs(wl, with_experts=False)
+    from sigmoid_top_routing_b200.device_inputs import bf16_tensor
+    x = bf16_tensor(inp.x_bits, "cuda")
+    wr = torch.from_numpy(inp.w_router).cuda()
+    b = torch.from_numpy(inp.expert_bias).cuda()
+    i_ref, w_ref = api.moe_route(x, None, wr, b, E=wl.E, k=wl.k, eps=wl.eps, scale=wl.router_scale)
+    # forward with dummy experts: only the router outputs are compared
+    W = api.ExpertWeights(act=0 if wl.act == "swiglu" else 1, fmt=0,
+                          w1=torch.zeros((wl.E, (2 if wl.act == "swiglu" else 1) * wl.I, wl.H),
+                                         dtype=torch.bfloat16, device="cuda"),
+                          w2=torch.zeros((wl.E, wl.H, wl.I), dtype=torch.bfloat16, device="cuda"))
+    _, i_fwd, w_fwd, _ = api.moe_forward(x, W, wr, b, E=wl.E, k=wl.k, I=wl.I, eps=wl.eps,
+                                         router_scale=wl.router_scale, out_scale=wl.out_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(i_fwd, i_ref)
+    assert torch.equal(w_fwd.view(torch.int32), w_ref.view(torch.int32))
