@@ -68,7 +68,8 @@ struct GemmParams {
     int* err;
 };
 
-template <int BN, int STAGES, int ASTAGE, int CSTAGE, int SBRING = (CSTAGE ? kSBDepth * 2 * 256 * 4 : 0)>
+template <int BN, int STAGES, int ASTAGE, int CSTAGE, bool USE_U,
+          int SBRING = (CSTAGE ? kSBDepth * 2 * 256 * 4 : 0)>
 struct Smem {
     static constexpr int kBStage = BN * 128;
     static constexpr size_t kA = 0;
@@ -80,9 +81,10 @@ struct Smem {
     static constexpr size_t kTileBase = kMisc + 16;                           // 257 ints
     static constexpr size_t kTok = kTileBase + 257 * 4;                       // BN ints (token of column)
     static constexpr size_t kTokW = kTok + BN * 4;                            // BN floats
-    static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats
-    static constexpr size_t kTrow = kU + 64 * 17 * 4;                         // BN ints (producer's token rows)
-    static constexpr size_t kSB = kTrow + BN * 4;                             // scale/bias ring (affine)
+    static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats (split SwiGLU)
+    static constexpr size_t kTrow = kU + (USE_U ? 64 * 17 * 4 : 0);          // BN ints (producer's token rows)
+    static constexpr size_t kCnt = kTrow + BN * 4;                            // 256 counts + 257 offsets
+    static constexpr size_t kSB = kCnt + 513 * 4 + 12;                        // scale/bias ring (affine)
     static constexpr size_t kEnd = kSB + SBRING;
     static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
 };
@@ -95,7 +97,7 @@ struct Tile {
 // weight-tile-major with the token tiles innermost, so the CTAs working at
 // one time share weight tiles in L2.
 template <int BN>
-MOE_DEV Tile decode_tile(int t, const int* base, int E, const int32_t* counts, const int32_t* offsets) {
+MOE_DEV Tile decode_tile(int t, const int* base, int E, const int* counts, const int* offsets) {
     int lo = 0, hi = E;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     // affine 4-bit: the A stage is written by the dequantisation warps from
     // packed codes (a quarter of the bf16 bytes) staged by TMA
     constexpr int kCStage = WFMT ? kAStage / 4 : 0;
-    using L = Smem<BN, STAGES, kAStage, kCStage>;
+    using L = Smem<BN, STAGES, kAStage, kCStage, MODE == kUpSwiglu && !kDual>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sA = sm + L::kA;
@@ -202,6 +204,8 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     float* s_tokw = reinterpret_cast<float*>(sm + L::kTokW);
     float* s_u = reinterpret_cast<float*>(sm + L::kU);
     int* s_trow = reinterpret_cast<int*>(sm + L::kTrow);
+    int* s_cnt = reinterpret_cast<int*>(sm + L::kCnt);      // plan counts and offsets, copied once
+    int* s_off = s_cnt + 256;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTmemCols = (kDual ? 4 : 2) * BN < 32 ? 32 : (kDual ? 4 : 2) * BN;
@@ -234,7 +238,17 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         tmem_relinquish();
         tc_fence_before();
     }
-    pdl_wait();   // the plan and (for down) h come from earlier kernels
+    // The up kernels follow the plan directly: they wait for it here.  The
+    // down kernel follows the up kernel and reads the plan (finished two
+    // launches earlier, read through L2) before waiting, so its weight tiles
+    // stream while the up kernel's last CTAs finish; only its producer waits,
+    // right before the first load of h.
+    if (MODE != kDown) pdl_wait();
+    for (int i = threadIdx.x; i < g.E; i += blockDim.x) {
+        s_cnt[i] = __ldcg(g.counts + i);
+        s_off[i] = __ldcg(g.offsets + i);
+    }
+    __syncthreads();
     // tile table: tiles of expert e = weight tiles x ceil(count / BN)
     const int fpt = (MODE == kUpSwiglu && !kDual) ? 64 : 128;   // output features per tile
     const int n_wt = (g.feats + fpt - 1) / fpt;
@@ -243,7 +257,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int local = 0;
         for (int j = 0; j < per; ++j) {
             const int e = lane * per + j;
-            if (e < g.E) local += n_wt * ((g.counts[e] + BN - 1) / BN);
+            if (e < g.E) local += n_wt * ((s_cnt[e] + BN - 1) / BN);
         }
         int incl = local;
 #pragma unroll
@@ -256,13 +270,17 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             const int e = lane * per + j;
             if (e < g.E) {
                 s_base[e] = run;
-                run += n_wt * ((g.counts[e] + BN - 1) / BN);
+                run += n_wt * ((s_cnt[e] + BN - 1) / BN);
             }
         }
         if (lane == 31) s_base[g.E] = incl;
     }
     __syncthreads();
     tc_fence_after();
+    // Every CTA of this persistent grid is resident by now, so the next kernel
+    // may launch: its CTAs take SMs as ours retire and run their prologue (the
+    // down kernel also its first weight loads) before waiting on this grid.
+    pdl_trigger();
     const uint32_t tmem_base = *s_tmem;
     const int total = s_base[g.E];
     const int nkb = g.K / kBK;
@@ -278,8 +296,29 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // several token tiles per weight tile the neighbours re-read it from L2
         const uint64_t pol_w = policy_evict_first();
         const bool hint_w = BN <= 32;
+        // down kernel: the first tile's first stages get their weight rows before
+        // the wait on the up kernel; their token rows (h) follow after it
+        int pre = 0;
+        if (MODE == kDown && blockIdx.x < total) {
+            const Tile tl = decode_tile<BN>(blockIdx.x, s_base, g.E, s_cnt, s_off);
+            pre = min(STAGES, nkb);
+            if (lane == 0) {
+                const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
+                const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
+                for (int kb = 0; kb < pre; ++kb) {   // fresh barriers: no empty wait needed
+                    mbar_arrive_expect_tx(&full[kb], (WFMT ? 0 : kAStage) + nbox * kBoxRows * 128);
+                    if (WFMT) {
+                        mbar_arrive_expect_tx(&cfull[kb], kCStage);
+                        tma_load_2d(sC + size_t(kb) * kCStage, &tmA, kb * 8, a_row, &cfull[kb]);
+                    } else {
+                        tma_load_2d(sA + size_t(kb) * kAStage, &tmA, kb * kBK, a_row, &full[kb]);
+                    }
+                }
+            }
+        }
+        if (MODE == kDown) pdl_wait();
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
             if (kGather) {
                 // token row of each B row (padding rows repeat the last token)
                 __syncwarp();
@@ -291,6 +330,20 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             }
             const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
             for (int kb = 0; kb < nkb; ++kb) {
+                if (pre > 0) {
+                    // weight rows already requested before the wait: add the token rows
+                    if (lane == 0) {
+                        const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
+                        unsigned char* b = sB + size_t(s) * L::kBStage;
+                        for (int j = 0; j < nbox; ++j)
+                            tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
+                    }
+                    --pre;
+                    issued_mask |= 1u << s;
+                    issued_par = (issued_par & ~(1u << s)) | (ph << s);
+                    if (++s == STAGES) { s = 0; ph ^= 1; }
+                    continue;
+                }
                 // all 32 lanes wait on the same phase; the decision is made warp-uniform
                 const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -348,7 +401,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-                const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+                const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
                 const int buf = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort)) { ok = false; break; }
@@ -406,7 +459,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // look-ahead iterator over this CTA's (tile, k-block) stages
         int at = blockIdx.x, akb = 0;
         Tile atl{};
-        if (at < total) atl = decode_tile<BN>(at, s_base, g.E, g.counts, g.offsets);
+        if (at < total) atl = decode_tile<BN>(at, s_base, g.E, s_cnt, s_off);
         auto issue = [&](int slot) {
             if (at < total) {
                 const size_t gr = grow(atl);
@@ -416,7 +469,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 if (++akb == nkb) {
                     akb = 0;
                     at += gridDim.x;
-                    if (at < total) atl = decode_tile<BN>(at, s_base, g.E, g.counts, g.offsets);
+                    if (at < total) atl = decode_tile<BN>(at, s_base, g.E, s_cnt, s_off);
                 }
             }
             cp_async_commit();
@@ -427,7 +480,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         uint32_t ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
             const size_t gr = grow(tl);
             for (int kb = 0; kb < nkb; ++kb) {
                 cp_async_wait<kSBDepth - 1>();               // this stage's scale/bias landed
@@ -472,7 +525,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int it = 0;
         bool dead = false;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, g.counts, g.offsets);
+            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
             const int buf = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             if (MODE == kDown) {
@@ -564,7 +617,6 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
     }
-    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -638,7 +690,7 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     if (e != cudaSuccess) return e;
     auto kern = k_gemm<MODE, BN, STAGES, WFMT>;
     constexpr int kA = (MODE == kUpSwiglu && BN >= 64) ? 2 * kARows : kARows;
-    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0>;   // + the scale/bias ring for affine
+    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0, MODE == kUpSwiglu && BN < 64>;   // + scale/bias ring (affine)
     static_assert(L::kBytes <= 227 * 1024, "shared memory of one CTA");
     const size_t smem = L::kBytes;
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
