@@ -91,13 +91,17 @@ struct Smem {
 
 struct Tile {
     int e, wt, tt, ntok, n, row0;
+    int kb0, kb1;            // k-blocks of this tile (a part of K when the reduction is split)
 };
 
 // Tile t -> (expert, weight tile, token tile).  Tiles of one expert run
 // weight-tile-major with the token tiles innermost, so the CTAs working at
 // one time share weight tiles in L2.
-template <int BN>
-MOE_DEV Tile decode_tile(int t, const int* base, int E, const int* counts, const int* offsets) {
+// With SPLIT, ks consecutive tile numbers share one output tile and each
+// takes a contiguous part of the nkb k-blocks.
+template <int BN, bool SPLIT>
+MOE_DEV Tile decode_tile(int tn, const int* base, int E, const int* counts, const int* offsets, int ks, int nkb) {
+    const int t = SPLIT ? tn / ks : tn;
     int lo = 0, hi = E;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -114,6 +118,14 @@ MOE_DEV Tile decode_tile(int t, const int* base, int E, const int* counts, const
     r.ntok = min(BN, c - r.tt * BN);
     r.n = (r.ntok + 15) & ~15;
     r.row0 = offsets[lo] + r.tt * BN;
+    if (SPLIT) {
+        const int part = tn - t * ks;
+        r.kb0 = part * nkb / ks;
+        r.kb1 = (part + 1) * nkb / ks;
+    } else {
+        r.kb0 = 0;
+        r.kb1 = nkb;
+    }
     return r;
 }
 
@@ -282,8 +294,17 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     // down kernel also its first weight loads) before waiting on this grid.
     pdl_trigger();
     const uint32_t tmem_base = *s_tmem;
-    const int total = s_base[g.E];
     const int nkb = g.K / kBK;
+    // The down projection's scatter-add is linear, so its reduction can be
+    // split: with less than ~4 waves of output tiles, K is cut into ks parts
+    // (>= 4 k-blocks each) whose partial sums all add into y_acc.
+    constexpr bool kSplit = MODE == kDown;
+    int ks = 1;
+    if (kSplit) {
+        const int t1 = max(s_base[g.E], 1);
+        ks = min(min(4, max(1, nkb / 4)), max(1, (4 * (int)gridDim.x + t1 - 1) / t1));
+    }
+    const int total = s_base[g.E] * ks;
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -300,25 +321,26 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // the wait on the up kernel; their token rows (h) follow after it
         int pre = 0;
         if (MODE == kDown && blockIdx.x < total) {
-            const Tile tl = decode_tile<BN>(blockIdx.x, s_base, g.E, s_cnt, s_off);
-            pre = min(STAGES, nkb);
+            const Tile tl = decode_tile<BN, kSplit>(blockIdx.x, s_base, g.E, s_cnt, s_off, ks, nkb);
+            pre = min(STAGES, tl.kb1 - tl.kb0);
             if (lane == 0) {
                 const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
                 const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
-                for (int kb = 0; kb < pre; ++kb) {   // fresh barriers: no empty wait needed
-                    mbar_arrive_expect_tx(&full[kb], (WFMT ? 0 : kAStage) + nbox * kBoxRows * 128);
+                for (int q = 0; q < pre; ++q) {      // fresh barriers: no empty wait needed
+                    const int kb = tl.kb0 + q;
+                    mbar_arrive_expect_tx(&full[q], (WFMT ? 0 : kAStage) + nbox * kBoxRows * 128);
                     if (WFMT) {
-                        mbar_arrive_expect_tx(&cfull[kb], kCStage);
-                        tma_load_2d(sC + size_t(kb) * kCStage, &tmA, kb * 8, a_row, &cfull[kb]);
+                        mbar_arrive_expect_tx(&cfull[q], kCStage);
+                        tma_load_2d(sC + size_t(q) * kCStage, &tmA, kb * 8, a_row, &cfull[q]);
                     } else {
-                        tma_load_2d(sA + size_t(kb) * kAStage, &tmA, kb * kBK, a_row, &full[kb]);
+                        tma_load_2d(sA + size_t(q) * kAStage, &tmA, kb * kBK, a_row, &full[q]);
                     }
                 }
             }
         }
         if (MODE == kDown) pdl_wait();
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
             if (kGather) {
                 // token row of each B row (padding rows repeat the last token)
                 __syncwarp();
@@ -329,7 +351,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 __syncwarp();
             }
             const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 if (pre > 0) {
                     // weight rows already requested before the wait: add the token rows
                     if (lane == 0) {
@@ -401,14 +423,14 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-                const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
+                const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
                 const int buf = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * (kDual ? 2 * BN : BN);
                 const uint32_t idesc = idesc_bf16(128, tl.n);
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
                     tc_fence_after();
                     if (kGather) fence_proxy_async_smem();   // cp.async-written rows -> tensor core
@@ -416,10 +438,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
-                        umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, (kb | kk) != 0);
+                        umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, kb != tl.kb0 || kk != 0);
                         if (kDual)   // up rows: the second 16 KB of the A stage, accumulator at + BN columns
                             umma_bf16(d + BN, ad + uint64_t((kARows >> 4) + kk * 2), bd + uint64_t(kk * 2), idesc,
-                                      (kb | kk) != 0);
+                                      kb != tl.kb0 || kk != 0);
                     }
                     umma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -459,17 +481,22 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // look-ahead iterator over this CTA's (tile, k-block) stages
         int at = blockIdx.x, akb = 0;
         Tile atl{};
-        if (at < total) atl = decode_tile<BN>(at, s_base, g.E, s_cnt, s_off);
+        if (at < total) {
+            atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
+            akb = atl.kb0;
+        }
         auto issue = [&](int slot) {
             if (at < total) {
                 const size_t gr = grow(atl);
                 const size_t gi = gr < nrows ? gr * G + akb : 0;
                 cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt), g.wscale + (gi & ~size_t(1)));
                 cp_async4(smem_u32(s_sb + (slot * 2 + 1) * 256 + dt), g.wbias + (gi & ~size_t(1)));
-                if (++akb == nkb) {
-                    akb = 0;
+                if (++akb == atl.kb1) {
                     at += gridDim.x;
-                    if (at < total) atl = decode_tile<BN>(at, s_base, g.E, s_cnt, s_off);
+                    if (at < total) {
+                        atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
+                        akb = atl.kb0;
+                    }
                 }
             }
             cp_async_commit();
@@ -480,9 +507,9 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         uint32_t ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
             const size_t gr = grow(tl);
-            for (int kb = 0; kb < nkb; ++kb) {
+            for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 cp_async_wait<kSBDepth - 1>();               // this stage's scale/bias landed
                 const uint32_t sw = s_sb[(slot * 2 + 0) * 256 + dt];
                 const uint32_t bw = s_sb[(slot * 2 + 1) * 256 + dt];
@@ -525,7 +552,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int it = 0;
         bool dead = false;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-            const Tile tl = decode_tile<BN>(t, s_base, g.E, s_cnt, s_off);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
             const int buf = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             if (MODE == kDown) {
