@@ -186,6 +186,25 @@ def cpu_oracle_rate(inp, budget_s: float):
     return done_tokens / t_used, f"{calls} oracle calls x {n} tokens of the workload ({t_used:.1f} s)", threads
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(v, dist, world: int, device, dtype):
+    """The maximum of v over all ranks.  Every rank calls it at the same
+    point (a collective); with one rank it returns v unchanged."""
+    if world <= 1:
+        return v
+    import torch
+    t = torch.tensor([v], device=device, dtype=dtype)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_rate(units_per_rank: float, world: int, seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank runs the same per-rank work)."""
+    return units_per_rank * world / seconds
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -349,10 +368,7 @@ def main():
         per = (time.perf_counter() - t0) / (B_steps * 4)
         K = int(max(B_steps, min(200000, 2.0 / per)))
         K = (K // B_steps) * B_steps
-    if world > 1:
-        kt = torch.tensor([K], device="cuda")
-        dist.all_reduce(kt, op=dist.ReduceOp.MAX)
-        K = int(kt.item())
+    K = int(max_over_ranks(K, dist, world, "cuda", torch.int64))
 
     sampler = ClockSampler(bus_id_of(torch, local))
     sampler.start()
@@ -378,18 +394,14 @@ def main():
     t_b = time.time()
     sampler.stop()
     ms = e0.elapsed_time(e1)
-    if world > 1:
-        mt = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(mt, op=dist.ReduceOp.MAX)
-        ms = float(mt.item())
+    ms = float(max_over_ranks(ms, dist, world, "cuda", torch.float64))
     assert api.moe_device_error(stream) == 0
 
     # up-kernel durations from the last block replay inside the timed region
     up_ms = [a.elapsed_time(b) for (a, b) in ev] if K >= B_steps else []
     clocks = sampler.summary(t_a - 0.5, t_b)
 
-    tokens = wl.T * K * world
-    value = tokens / (ms / 1e3)
+    value = job_rate(wl.T * K, world, ms / 1e3)
     pk, pk_kind = peaks()
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
@@ -472,11 +484,8 @@ def main():
         for j in range(n_e2e):
             host_call(Ws[j % n_sets])
         el = time.perf_counter() - t0
-        if world > 1:
-            tt = torch.tensor([el], device="cuda", dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            el = float(tt.item())
-        line["e2e"] = {"value": wl.T * n_e2e * world / el, "unit": "tokens/s",
+        el = float(max_over_ranks(el, dist, world, "cuda", torch.float64))
+        line["e2e"] = {"value": job_rate(wl.T * n_e2e, world, el), "unit": "tokens/s",
                        "h2d_bytes_per_step": wl.T * wl.H * 2, "d2h_bytes_per_step": wl.T * wl.H * 2,
                        "steps": n_e2e, "timing": "host wall clock around synchronous moe_forward_host calls"}
 

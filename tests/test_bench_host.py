@@ -1,0 +1,80 @@
+"""Host-side logic of bench.py for N > 1 ranks, run as two gloo ranks on CPU.
+
+The block shards by tokens with no exchange step, so N GPUs run N independent
+replicas; what ranks share is the bookkeeping: every rank agrees on the step
+count (maximum over ranks), the timed duration is the slowest rank's, and the
+reported value is the tokens all ranks processed over that duration.
+"""
+import importlib.util
+import os
+import socket
+import sys
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist          # noqa: E402
+import torch.multiprocessing as mp        # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        b = _bench()
+        K = int(b.max_over_ranks(100 + 7 * rank, dist, world, "cpu", torch.int64))
+        ms = float(b.max_over_ranks(10.0 + rank * 2.5, dist, world, "cpu", torch.float64))
+        value = b.job_rate(8 * K, world, ms / 1e3)
+        q.put((rank, K, ms, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_steps_and_slowest_time():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    for rank, K, ms, value in got:
+        assert K == 107                  # the larger step count
+        assert ms == pytest.approx(12.5)  # the slowest rank
+        assert value == pytest.approx(8 * 107 * world / 12.5e-3)
+
+
+def test_single_rank_is_a_no_op():
+    b = _bench()
+    assert b.max_over_ranks(3.5, None, 1, "cpu", torch.float64) == 3.5
+    assert b.job_rate(1000, 1, 0.5) == 2000
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
+    b = _bench()
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2"])
+    args = b.parse()
+    assert b.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
