@@ -74,8 +74,12 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1 } moe_wfmt;
 
 /* Which expert kernels moe_experts / moe_forward use (process-wide). */
 typedef enum {
-    MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM at every T */
-    MOE_DISPATCH_GEMV = 1, /* the CUDA-core weight-streaming grouped GEMV (bf16 only) */
+    MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM, except affine
+                              4-bit experts at <= 8 routed pairs per expert on average
+                              (T*k <= 8*E, H and I <= 8192), which take the
+                              register-dequant GEMV */
+    MOE_DISPATCH_GEMV = 1, /* the weight-streaming grouped GEMV (bf16: CUDA cores; affine
+                              4-bit: codes dequantised in registers, m16n8k16 dot products) */
     MOE_DISPATCH_GEMM = 2  /* the tcgen05 grouped GEMM */
 } moe_dispatch;
 

@@ -75,6 +75,13 @@ cudaError_t launch_plan(const PlanArgs& a, bool pdl, cudaStream_t s, int* n_laun
 size_t plan_scratch_ints(int P, int E);
 cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// Affine 4-bit GEMV (codes dequantised in registers); launch_gemv_up/down
+// route fmt == 1 here.
+cudaError_t launch_gemv_affine_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemv_affine_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// MOE_DISPATCH_AUTO's choice: the GEMV for affine 4-bit experts with at most
+// this many routed pairs per expert on average, the tcgen05 GEMM otherwise.
+constexpr int kAffineGemvMaxPairsPerExpert = 8;
 // The tcgen05 grouped GEMMs (cudaErrorNotSupported where a format has none).
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);

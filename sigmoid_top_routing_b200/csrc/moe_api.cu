@@ -171,9 +171,16 @@ int current_dispatch() {
     return g_dispatch;
 }
 
-// The tcgen05 grouped GEMM serves every token count (its token tiles shrink
-// to N = 16 for decode batches); the CUDA-core GEMV stays selectable.
-bool use_gemv(const moe_dims*) { return current_dispatch() == MOE_DISPATCH_GEMV; }
+// bf16: the tcgen05 grouped GEMM serves every token count (its token tiles
+// shrink to 32 for decode batches); the CUDA-core GEMV stays selectable.
+// Affine 4-bit: up to a few pairs per expert the register-dequant GEMV streams
+// the codes faster than the GEMM's shared-memory dequant pipeline.
+bool use_gemv(const moe_dims* d, int32_t fmt) {
+    const int mode = current_dispatch();
+    if (mode != MOE_DISPATCH_AUTO) return mode == MOE_DISPATCH_GEMV;
+    return fmt == MOE_W_AFFINE4_G64 && d->H <= 8192 && d->I <= 8192 &&
+           (size_t)d->T * d->k <= (size_t)kAffineGemvMaxPairsPerExpert * d->E;
+}
 
 ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* topk_w,
                             const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
@@ -239,7 +246,7 @@ struct Seq {
 };
 
 moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
-    const bool gemv = use_gemv(d);
+    const bool gemv = use_gemv(d, a.fmt);
     cudaError_t e;
     if (!gemv && gemm_needs_xs(a)) {
         // token rows in plan order for the wide up tiles (part of the plan's data movement)

@@ -1,7 +1,8 @@
-"""Parity of the MLX-style affine 4-bit expert path (codes dequantised on chip
-into the tcgen05 operand) with the float64 oracle, which dequantises the same
-codes exactly.  Gate: rel-L2 <= 3e-2 (the weights are rounded once to bf16
-on chip, the oracle keeps them exact)."""
+"""Parity of the MLX-style affine 4-bit expert paths with the float64 oracle,
+which dequantises the same codes exactly.  Two paths: the tcgen05 GEMM (codes
+dequantised on chip into its shared-memory operand, weights rounded once to
+bf16) and the decode GEMV (codes dequantised in registers, scale and bias
+applied in fp32 per group).  Gate: rel-L2 <= 3e-2."""
 import dataclasses
 
 import numpy as np
@@ -37,10 +38,29 @@ def test_affine4_relu2_small(api):
     _check_all(inp, run_forward(api, inp))
 
 
+@pytest.mark.parametrize("path", ["auto", "gemm", "gemv"])
 @pytest.mark.parametrize("T", [1, 8, 64])
-def test_affine4_decode_sizes(api, T):
+def test_affine4_decode_sizes(api, T, path):
+    from sigmoid_top_routing_b200 import abi
+    d = {"auto": abi.MOE_DISPATCH_AUTO, "gemm": abi.MOE_DISPATCH_GEMM, "gemv": abi.MOE_DISPATCH_GEMV}[path]
     inp = inputs_of(G.WORKLOADS[f"affine4_t{T}"])
-    _check_all(inp, run_forward(api, inp))
+    _check_all(inp, run_forward(api, inp, dispatch=d))
+
+
+def test_affine4_gemv_token_chunks_and_short_k(api):
+    """GEMV with more than 8 tokens per expert (several token chunks per row
+    block) and H = 128 (two groups of 64: most warps get no K slice)."""
+    from sigmoid_top_routing_b200 import abi
+    wl = G.Workload("a4_small", T=33, H=128, E=8, k=4, I=64, fmt="affine4")
+    inp = inputs_of(wl)
+    _check_all(inp, run_forward(api, inp, dispatch=abi.MOE_DISPATCH_GEMV))
+
+
+def test_affine4_gemv_relu2(api):
+    from sigmoid_top_routing_b200 import abi
+    wl = G.Workload("a4_relu2", T=40, H=256, E=16, k=6, I=192, act="relu2", fmt="affine4", out_scale=2.5)
+    inp = inputs_of(wl)
+    _check_all(inp, run_forward(api, inp, dispatch=abi.MOE_DISPATCH_GEMV))
 
 
 def test_affine4_t512(api):
