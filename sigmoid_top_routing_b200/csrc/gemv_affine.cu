@@ -79,8 +79,6 @@ MOE_DEV uint32_t ld_u16(const uint16_t* p) {
     return v;
 }
 
-MOE_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
-
 MOE_DEV void cp_async16(void* smem, const void* gmem) {
     const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
