@@ -435,12 +435,20 @@ def main():
 
     # in-situ time of each stage: graphs of B steps with events around one stage
     if not args.no_stages:
-        names = [(abi.MOE_STAGE_ROUTE, "route"), (abi.MOE_STAGE_PLAN, "plan"), (abi.MOE_STAGE_UP, "up"),
+        names = [(abi.MOE_STAGE_ROUTE, "route"), (abi.MOE_STAGE_PLAN, "plan"),
+                 (abi.MOE_STAGE_GATHER, "gather"), (abi.MOE_STAGE_UP, "up"),
                  (abi.MOE_STAGE_DOWN, "down"), (abi.MOE_STAGE_FINAL, "finalize")]
+        # the library's AUTO choice: affine 4-bit experts at <= 8 pairs per expert take the GEMV
+        gemv_path = args.dispatch == "gemv" or (
+            args.dispatch == "auto" and wl.fmt != "bf16" and wl.T * wl.k <= 8 * wl.E
+            and wl.H <= 8192 and wl.I <= 8192)
         stage_us = {}
         for sid, nm in names:
             if sid == abi.MOE_STAGE_PLAN and wl.T <= 32:
                 stage_us[nm] = "fused into route"     # one CTA routes and plans at T <= 32
+                continue
+            if sid == abi.MOE_STAGE_GATHER and gemv_path:
+                stage_us[nm] = "not launched (GEMV path)"
                 continue
             evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(B_steps)]

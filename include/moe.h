@@ -195,7 +195,8 @@ typedef enum {
     MOE_STAGE_PLAN = 1,    /* the plan kernel (fused into the router for T <= 32) */
     MOE_STAGE_UP = 2,      /* the expert up-projection + activation kernel */
     MOE_STAGE_DOWN = 3,    /* the expert down-projection + weighted scatter kernel */
-    MOE_STAGE_FINAL = 4    /* the output scale + bf16 rounding kernel */
+    MOE_STAGE_FINAL = 4,   /* the output scale + bf16 rounding kernel */
+    MOE_STAGE_GATHER = 5   /* the copy of token rows into plan order (tcgen05 GEMM path) */
 } moe_stage;
 
 /* One-shot timing hook for the calling thread: the next moe_forward /

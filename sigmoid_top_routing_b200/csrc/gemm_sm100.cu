@@ -22,8 +22,8 @@
 // only on its row and expert; changed for sm_100a: TMA, tcgen05, TMEM.
 //
 // Warp roles (192 threads, one CTA per SM, persistent over tiles):
-//   warp 0      producer: TMA for weights; token rows gathered with cp.async
-//               (up) or TMA (down, h is contiguous in plan order)
+//   warp 0      producer: TMA for weights and for token rows (up: xs, the
+//               rows gathered in plan order by k_gather_rows; down: h)
 //   warp 1      TMEM owner and MMA issuer (one thread)
 //   warps 2..5  epilogue (TMEM lanes 32 * (warp % 4) ...)
 // Every mbarrier wait is bounded; on expiry the kernel records error code 2,
@@ -82,8 +82,7 @@ struct Smem {
     static constexpr size_t kTok = kTileBase + 257 * 4;                       // BN ints (token of column)
     static constexpr size_t kTokW = kTok + BN * 4;                            // BN floats
     static constexpr size_t kU = kTokW + BN * 4;                              // 64 x 17 floats (split SwiGLU)
-    static constexpr size_t kTrow = kU + (USE_U ? 64 * 17 * 4 : 0);          // BN ints (producer's token rows)
-    static constexpr size_t kCnt = kTrow + BN * 4;                            // 256 counts + 257 offsets
+    static constexpr size_t kCnt = kU + (USE_U ? 64 * 17 * 4 : 0);           // 256 counts + 257 offsets
     static constexpr size_t kSB = kCnt + 513 * 4 + 12;                        // scale/bias ring (affine)
     static constexpr size_t kEnd = kSB + SBRING;
     static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
@@ -133,12 +132,6 @@ MOE_DEV Tile decode_tile(int tn, const int* base, int E, const int* counts, cons
 // rounded to bf16); NaN propagates, g -> -inf gives -0 * u.
 MOE_DEV float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-MOE_DEV void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-MOE_DEV void cp_async_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 // Dequantise 16-byte chunks [c0, c0 + NC) of one 128-byte A row (8 affine
 // 4-bit codes per chunk, one group per row per k-block) into the 128-byte-
@@ -215,17 +208,13 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     int* s_tok = reinterpret_cast<int*>(sm + L::kTok);
     float* s_tokw = reinterpret_cast<float*>(sm + L::kTokW);
     float* s_u = reinterpret_cast<float*>(sm + L::kU);
-    int* s_trow = reinterpret_cast<int*>(sm + L::kTrow);
     int* s_cnt = reinterpret_cast<int*>(sm + L::kCnt);      // plan counts and offsets, copied once
     int* s_off = s_cnt + 256;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTmemCols = (kDual ? 4 : 2) * BN < 32 ? 32 : (kDual ? 4 : 2) * BN;
-    // up: 32 producer lanes gather token rows with cp.async, + 1 expect_tx arrive
-    // decode-width up tiles gather token rows from x with cp.async (32 lanes + the
-    // expect_tx arrive); wider tiles take rows of xs (up) or h (down) by TMA
-    constexpr bool kGather = MODE != kDown && BN <= 32;
-    constexpr uint32_t kFullCount = (kGather ? 33 : 1) + (WFMT ? 256 : 0);   // + 256 dequant threads
+    // token rows come by TMA: from xs (up, gathered in plan order) or h (down)
+    constexpr uint32_t kFullCount = 1 + (WFMT ? 256 : 0);   // expect_tx arrive + 256 dequant threads
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -243,7 +232,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
-        if (!kGather) tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, kTmemCols);
@@ -341,15 +330,6 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         if (MODE == kDown) pdl_wait();
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
-            if (kGather) {
-                // token row of each B row (padding rows repeat the last token)
-                __syncwarp();
-                for (int r = lane; r < tl.n; r += 32) {
-                    const int rr = r < tl.ntok ? r : tl.ntok - 1;
-                    s_trow[r] = g.perm[tl.row0 + rr] / g.k;
-                }
-                __syncwarp();
-            }
             const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
             for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 if (pre > 0) {
@@ -371,7 +351,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 if (lane == 0) {
                     const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
-                    const uint32_t bytes = (WFMT ? 0 : kAStage) + (kGather ? 0 : nbox * kBoxRows * 128);
+                    const uint32_t bytes = (WFMT ? 0 : kAStage) + nbox * kBoxRows * 128;
                     mbar_arrive_expect_tx(&full[s], bytes);
                     if (WFMT) mbar_arrive_expect_tx(&cfull[s], kCStage);
                     // bf16: weight rows straight into the A stage; affine: codes into the staging area
@@ -387,21 +367,9 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                         tma_load_2d(a, &tmA, ax, a_row, abar);
                         if (MODE == kUpSwiglu) tma_load_2d(a + kHalf, &tmA, ax, a_row + g.I, abar);
                     }
-                    if (!kGather) {
-                        unsigned char* b = sB + size_t(s) * L::kBStage;
-                        for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
-                    }
-                }
-                if (kGather) {
-                    // gather: 8 lanes cover one 128-byte row slice, 4 rows per instruction;
-                    // row r, 16-byte chunk c lands at the swizzled (r, c ^ (r & 7))
-                    const uint32_t b = smem_u32(sB + size_t(s) * L::kBStage);
-                    const int c = lane & 7;
-                    const unsigned char* xb = reinterpret_cast<const unsigned char*>(g.x) + kb * 128 + c * 16;
-                    for (int r = lane >> 3; r < tl.n; r += 4)
-                        cp_async16(b + r * 128 + ((c ^ (r & 7)) << 4), xb + (size_t)s_trow[r] * g.H * 2);
-                    cp_async_arrive(&full[s]);
+                    unsigned char* b = sB + size_t(s) * L::kBStage;
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
                 }
                 issued_mask |= 1u << s;
                 issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -433,7 +401,6 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
                     tc_fence_after();
-                    if (kGather) fence_proxy_async_smem();   // cp.async-written rows -> tensor core
                     const uint64_t ad = sdesc_sw128(smem_u32(sA + size_t(s) * kAStage));
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
 #pragma unroll
@@ -709,10 +676,8 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
         e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, b_box);
-    } else if (BN > 32) {
-        e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, b_box);   // rows gathered in plan order
     } else {
-        e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, 16);          // unused (cp.async gather)
+        e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, b_box);   // rows gathered in plan order
     }
     if (e != cudaSuccess) return e;
     auto kern = k_gemm<MODE, BN, STAGES, WFMT>;
@@ -779,7 +744,6 @@ __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict_
 
 }  // namespace
 
-bool gemm_needs_xs(const ExpertArgs& a) { return pick_bn(a) > 32; }
 
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const int P = a.T * a.k;

@@ -85,9 +85,8 @@ constexpr int kAffineGemvMaxPairsPerExpert = 8;
 // The tcgen05 grouped GEMMs (cudaErrorNotSupported where a format has none).
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
-// Wide token tiles take the up GEMM's token rows from xs (plan order), filled
-// by launch_gather_x; decode-width tiles gather from x themselves.
-bool gemm_needs_xs(const ExpertArgs& a);
+// The up GEMM takes its token rows by TMA from xs, the rows of x in plan
+// order, filled by launch_gather_x before it.
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s);

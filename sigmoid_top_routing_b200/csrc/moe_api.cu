@@ -248,9 +248,9 @@ struct Seq {
 moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
     const bool gemv = use_gemv(d, a.fmt);
     cudaError_t e;
-    if (!gemv && gemm_needs_xs(a)) {
-        // token rows in plan order for the wide up tiles (part of the plan's data movement)
-        e = q.stage(-1, [&](int*) { return launch_gather_x(a, true, q.s); });
+    if (!gemv) {
+        // token rows in plan order for the up GEMM's TMA (part of the plan's data movement)
+        e = q.stage(MOE_STAGE_GATHER, [&](int*) { return launch_gather_x(a, true, q.s); });
         if (e != cudaSuccess) return cuda_fail(e, "gather token rows");
     }
     e = q.stage(MOE_STAGE_UP, [&](int*) {
@@ -486,7 +486,7 @@ moe_status moe_profile_hook(void* ev_begin, void* ev_end, int32_t stage) {
         g_hook = Hook{};
         return MOE_OK;
     }
-    if (stage < MOE_STAGE_ROUTE || stage > MOE_STAGE_FINAL) return fail(MOE_ERR_UNSUPPORTED, "stage %d", stage);
+    if (stage < MOE_STAGE_ROUTE || stage > MOE_STAGE_GATHER) return fail(MOE_ERR_UNSUPPORTED, "stage %d", stage);
     g_hook.begin = static_cast<cudaEvent_t>(ev_begin);
     g_hook.end = static_cast<cudaEvent_t>(ev_end);
     g_hook.stage = stage;
