@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--dispatch", default="auto", choices=["auto", "gemv", "gemm"],
                     help="expert kernels: the library's choice, the grouped GEMV or the tcgen05 GEMM")
+    ap.add_argument("--combine", default="atomic", choices=["atomic", "ordered"],
+                    help="combine of the k expert outputs: fp32 atomics, or slot-ordered (reproducible)")
     ap.add_argument("--profile", action="store_true",
                     help="only W + K plain forward calls (for a profiler); prints the work model")
     ap.add_argument("--no-e2e", action="store_true")
@@ -273,6 +275,7 @@ def main():
     api.load()
 
     wl = G.WORKLOADS[args.workload]
+    api.moe_set_combine({"atomic": abi.MOE_COMBINE_ATOMIC, "ordered": abi.MOE_COMBINE_ORDERED}[args.combine])
     api.moe_set_dispatch({"auto": abi.MOE_DISPATCH_AUTO, "gemv": abi.MOE_DISPATCH_GEMV,
                           "gemm": abi.MOE_DISPATCH_GEMM}[args.dispatch])
     inp = G.make_inputs(wl)
@@ -409,7 +412,8 @@ def main():
             "config": dict(config_of(wl), l2=f"inputs larger than L2: {n_sets} weight copies rotated "
                                              f"({n_sets * all_w / 1e9:.2f} GB, {wm['active_experts']} "
                                              f"active experts per step)",
-                           graphs=f"CUDA graphs of {B_steps} steps", expert_kernels=args.dispatch),
+                           graphs=f"CUDA graphs of {B_steps} steps", expert_kernels=args.dispatch,
+                           combine=args.combine),
             "gpu_launches": launches_per_step * K, "clocks": clocks}
 
     # roofline of the dominant kernel (expert up-projection + activation)

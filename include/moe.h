@@ -132,7 +132,8 @@ typedef struct {
 
 /* Byte offsets of the regions inside the workspace (for inspection/tests). */
 typedef struct {
-    size_t y_acc;   /* fp32 (T, H): the unscaled routed sum */
+    size_t y_acc;   /* fp32 (T, H): the unscaled routed sum; (P, H) weighted slot outputs
+                       under MOE_COMBINE_ORDERED */
     size_t h;       /* bf16 (P, I): activations in plan order */
     size_t xs;      /* bf16 (P, H): token rows gathered in plan order (wide token tiles) */
     size_t scratch; /* plan and scheduler scratch */
@@ -239,6 +240,21 @@ MOE_API moe_status moe_forward_static(const void* x, const float* logits, const 
 
 /* Process-wide choice of expert kernels (moe_dispatch); returns the old one. */
 MOE_API int32_t moe_set_dispatch(int32_t mode);
+
+/* How the weighted expert outputs of a token are combined (process-wide).
+ *   MOE_COMBINE_ATOMIC  (default): the down projection adds w_j * o_j into the
+ *     fp32 accumulator y_acc (T, H) with atomic reductions; the order of the
+ *     k additions, and so the last bits of y, can vary from run to run.
+ *   MOE_COMBINE_ORDERED: the down projection stores w_j * o_j per plan slot
+ *     (fp32 (P, H), in the workspace's y_acc region) and the finalize sums a
+ *     token's k slots in slot order j = 0..k-1, then scales once.  y is then
+ *     bitwise reproducible, and for bf16 experts a token's y does not depend
+ *     on the other tokens of the batch (the router already has a fixed
+ *     summation order).  The workspace is larger (P * H * 4 bytes for that
+ *     region): query moe_workspace_bytes after setting the mode.  Not used by
+ *     moe_forward_static. */
+typedef enum { MOE_COMBINE_ATOMIC = 0, MOE_COMBINE_ORDERED = 1 } moe_combine;
+MOE_API int32_t moe_set_combine(int32_t mode);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code = 0 when no kernel reported an error.  Codes:

@@ -20,6 +20,7 @@ STATUS_NAMES = ["MOE_OK", "MOE_ERR_NULL", "MOE_ERR_SHAPE", "MOE_ERR_ALIGN", "MOE
 MOE_ACT_SWIGLU, MOE_ACT_RELU2 = 0, 1
 MOE_W_BF16, MOE_W_AFFINE4_G64 = 0, 1
 MOE_DISPATCH_AUTO, MOE_DISPATCH_GEMV, MOE_DISPATCH_GEMM = 0, 1, 2
+MOE_COMBINE_ATOMIC, MOE_COMBINE_ORDERED = 0, 1
 MOE_STAGE_ROUTE, MOE_STAGE_PLAN, MOE_STAGE_UP, MOE_STAGE_DOWN, MOE_STAGE_FINAL, MOE_STAGE_GATHER = range(6)
 MOE_TILE_M = 128
 
@@ -65,6 +66,7 @@ PROTOTYPES = {
     "moe_profile_hook": (c_int32, [c_void_p, c_void_p, c_int32]),
     "moe_last_launch_count": (c_int32, []),
     "moe_set_dispatch": (c_int32, [c_int32]),
+    "moe_set_combine": (c_int32, [c_int32]),
     "moe_device_error": (c_int32, [POINTER(c_int32), c_void_p]),
     "moe_last_error": (c_char_p, []),
     "moe_version": (c_char_p, []),

@@ -17,7 +17,7 @@ from .abi import check, load
 
 __all__ = [
     "ExpertWeights", "Plan", "moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_plan",
-    "moe_experts", "moe_forward", "moe_forward_host", "moe_set_dispatch", "moe_device_error",
+    "moe_experts", "moe_forward", "moe_forward_host", "moe_set_dispatch", "moe_set_combine", "moe_device_error",
     "moe_last_error", "moe_version", "new_plan", "new_workspace", "dims", "moe_profile_hook",
     "moe_last_launch_count",
 ]
@@ -185,6 +185,10 @@ def moe_last_launch_count() -> int:
 
 def moe_set_dispatch(mode: int) -> int:
     return int(load().moe_set_dispatch(mode))
+
+
+def moe_set_combine(mode: int) -> int:
+    return int(load().moe_set_combine(mode))
 
 
 def moe_device_error(stream=None) -> int:

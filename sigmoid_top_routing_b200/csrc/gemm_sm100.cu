@@ -58,7 +58,8 @@ struct GemmParams {
     const float* topk_w;
     const uint16_t* x;       // (T, H) token rows (up)
     uint16_t* h;             // (P, I) activations in plan order (written by up, read by down)
-    float* y_acc;            // (T, H) (down)
+    float* y_acc;            // (T, H) (down), or (P, H) per-slot outputs when ordered
+    int ordered;             // down: store w * o per plan slot instead of adding into y_acc
     int E, k, H, I;
     int K;                   // reduction length: H (up) or I (down)
     int rows_per_expert;     // rows of the A tensor per expert: 2I, I or H
@@ -289,7 +290,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     // (>= 4 k-blocks each) whose partial sums all add into y_acc.
     constexpr bool kSplit = MODE == kDown;
     int ks = 1;
-    if (kSplit) {
+    if (kSplit && !g.ordered) {   // ordered: each slot row is stored once, whole
         const int t1 = max(s_base[g.E], 1);
         ks = min(min(4, max(1, nkb / 4)), max(1, (4 * (int)gridDim.x + t1 - 1) / t1));
     }
@@ -554,7 +555,11 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
-                            if (c < tl.ntok) red_add_f32(g.y_acc + (size_t)s_tok[c] * g.H + f, s_tokw[c] * v[i]);
+                            if (c >= tl.ntok) continue;
+                            if (g.ordered)
+                                __stcg(g.y_acc + (size_t)(tl.row0 + c) * g.H + f, s_tokw[c] * v[i]);
+                            else
+                                red_add_f32(g.y_acc + (size_t)s_tok[c] * g.H + f, s_tokw[c] * v[i]);
                         }
                     }
                 } else if (MODE == kUpRelu2) {
@@ -707,6 +712,7 @@ GemmParams params(const ExpertArgs& a, bool up) {
     g.x = a.x;
     g.h = a.h;
     g.y_acc = a.y_acc;
+    g.ordered = a.ordered;
     g.E = a.E;
     g.k = a.k;
     g.H = a.H;

@@ -167,7 +167,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_gemv_down(ExpertArgs a) {
             for (int m = 0; m < kTokGroup; ++m) {
                 if (m < mt && lane == m) {
                     const float wv = a.topk_w[pm[m]];
-                    atomicAdd(a.y_acc + (size_t)(pm[m] / a.k) * H + n, wv * so[m]);
+                    if (a.ordered)
+                        a.y_acc[(size_t)(off + m0 + m) * H + n] = wv * so[m];
+                    else
+                        atomicAdd(a.y_acc + (size_t)(pm[m] / a.k) * H + n, wv * so[m]);
                 }
             }
         }
@@ -191,6 +194,32 @@ __global__ void __launch_bounds__(256) k_finalize(ExpertArgs a) {
         o.z = pack_bf16x2(sc * v1.x, sc * v1.y);
         o.w = pack_bf16x2(sc * v1.z, sc * v1.w);
         dst[i] = o;
+    }
+    pdl_trigger();
+}
+
+// Ordered combine: y[t] = bf16_rn(out_scale * (sum over j = 0..k-1, in that
+// order, of the slot row inv[t * k + j])); the rows already carry w_j.
+__global__ void __launch_bounds__(256) k_finalize_ordered(ExpertArgs a) {
+    pdl_wait();
+    const size_t n4 = (size_t)a.T * a.H / 4;
+    const int h4 = a.H / 4;
+    const float sc = a.out_scale;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const int t = (int)(i / h4), c = (int)(i - (size_t)t * h4);
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < a.k; ++j) {
+            const int slot = a.inv[(size_t)t * a.k + j];
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(a.y_acc + (size_t)slot * a.H) + c);
+            s.x += v.x;
+            s.y += v.y;
+            s.z += v.z;
+            s.w += v.w;
+        }
+        uint2 o;
+        o.x = pack_bf16x2(sc * s.x, sc * s.y);
+        o.y = pack_bf16x2(sc * s.z, sc * s.w);
+        reinterpret_cast<uint2*>(a.y)[i] = o;
     }
     pdl_trigger();
 }
@@ -224,6 +253,11 @@ cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const size_t n8 = (size_t)a.T * a.H / 8;
     if (n8 == 0) return cudaSuccess;
     const DeviceInfo& di = device_info();
+    if (a.ordered) {
+        const size_t n4 = n8 * 2;
+        size_t blocks = (n4 + 255) / 256, cap = (size_t)di.sm_count * 8;
+        return launch_k(k_finalize_ordered, dim3((unsigned)(blocks < cap ? blocks : cap)), dim3(256), 0, s, pdl, a);
+    }
     size_t blocks = (n8 + 255) / 256;
     size_t cap = (size_t)di.sm_count * 8;
     return launch_k(k_finalize, dim3((unsigned)(blocks < cap ? blocks : cap)), dim3(256), 0, s, pdl, a);

@@ -241,9 +241,15 @@ __global__ void __launch_bounds__(kA4Warps * 32, 4) k_gemv_a4(ExpertArgs a) {
                 } else {
                     const int pair = a.perm[slot];
                     const float wt = a.topk_w[pair];
-                    float* yrow = a.y_acc + (size_t)(pair / a.k) * a.H + rb * 16 + g;
-                    atomicAdd(yrow, wt * acc[jn]);
-                    atomicAdd(yrow + 8, wt * acc[2 + jn]);
+                    if (a.ordered) {
+                        float* orow = a.y_acc + (size_t)slot * a.H + rb * 16 + g;
+                        orow[0] = wt * acc[jn];
+                        orow[8] = wt * acc[2 + jn];
+                    } else {
+                        float* yrow = a.y_acc + (size_t)(pair / a.k) * a.H + rb * 16 + g;
+                        atomicAdd(yrow, wt * acc[jn]);
+                        atomicAdd(yrow + 8, wt * acc[2 + jn]);
+                    }
                 }
             }
         }

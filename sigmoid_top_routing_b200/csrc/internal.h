@@ -41,6 +41,7 @@ struct ExpertArgs {
     const int32_t* counts;
     const int32_t* offsets;
     const int32_t* perm;
+    const int32_t* inv;      // pair t * k + j -> plan slot (ordered combine)
     const int32_t* tiles;
     int T, H, E, k, I;
     int act;                 // 0 swiglu, 1 relu2
@@ -53,7 +54,8 @@ struct ExpertArgs {
     const uint16_t* w2_bias;
     uint16_t* h;             // (P, I) bf16 in plan order
     uint16_t* xs;            // (P, H) bf16 gathered rows (GEMM path)
-    float* y_acc;            // (T, H) fp32
+    float* y_acc;            // (T, H) fp32, or (P, H) weighted slot outputs when ordered
+    int ordered;             // 1: down stores w * o per plan slot; finalize sums slots in order
     uint16_t* y;             // (T, H) bf16
     float out_scale;
     int* err;

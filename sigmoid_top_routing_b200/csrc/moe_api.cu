@@ -47,6 +47,12 @@ struct Hook {
 thread_local Hook g_hook;
 std::mutex g_dispatch_mu;
 int g_dispatch = MOE_DISPATCH_AUTO;
+int g_combine = MOE_COMBINE_ATOMIC;   // guarded by g_dispatch_mu
+
+bool combine_ordered() {
+    std::lock_guard<std::mutex> lock(g_dispatch_mu);
+    return g_combine == MOE_COMBINE_ORDERED;
+}
 
 moe_status fail(moe_status st, const char* fmt, ...) {
     char buf[512];
@@ -88,8 +94,8 @@ moe_status check_fmt(int32_t fmt) {
 void layout(const moe_dims* d, moe_ws_layout* L) {
     const size_t T = d->T, H = d->H, E = d->E, P = (size_t)d->T * d->k, I = d->I;
     size_t off = 0;
-    L->y_acc = off;
-    off = align256(off + T * H * 4);
+    L->y_acc = off;       // (T, H) sums, or (P, H) slot outputs for the ordered combine
+    off = align256(off + (combine_ordered() ? P : T) * H * 4);
     L->h = off;
     off = align256(off + P * I * 2);
     L->xs = off;          // token rows gathered in plan order (wide token tiles)
@@ -191,6 +197,7 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.counts = plan->counts;
     a.offsets = plan->offsets;
     a.perm = plan->perm;
+    a.inv = plan->inv;
     a.tiles = plan->tiles;
     a.T = d->T;
     a.H = d->H;
@@ -208,6 +215,7 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.h = v.h;
     a.xs = v.xs;
     a.y_acc = v.y_acc;
+    a.ordered = combine_ordered() ? 1 : 0;
     a.y = static_cast<uint16_t*>(y);
     a.out_scale = out_scale;
     a.err = device_info().err_word;
@@ -370,10 +378,12 @@ moe_status moe_experts(const void* x, const moe_plan_t* plan, const float* topk_
     WsView v;
     if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
     Seq q{reinterpret_cast<cudaStream_t>(stream)};
-    cudaError_t e = launch_zero(v.y_acc, (size_t)d->T * d->H, true, q.s);
-    if (e != cudaSuccess) return cuda_fail(e, "zero y_acc");
-    q.n = 1;
     const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    if (!a.ordered) {   // the ordered combine writes every slot row: nothing to clear
+        cudaError_t e = launch_zero(v.y_acc, (size_t)d->T * d->H, true, q.s);
+        if (e != cudaSuccess) return cuda_fail(e, "zero y_acc");
+        q.n = 1;
+    }
     if ((st = run_experts(q, a, d)) != MOE_OK) return st;
     g_launches = q.n;
     return MOE_OK;
@@ -417,7 +427,7 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
     r.perm = plan->perm;
     r.inv = plan->inv;
     r.tiles = plan->tiles;
-    r.zero_ptr = v.y_acc;              // the router also clears the fp32 accumulator
+    r.zero_ptr = combine_ordered() ? nullptr : v.y_acc;   // the router also clears the accumulator
     r.zero_count = (size_t)d->T * d->H;
     r.err = device_info().err_word;
     const bool fuse = d->T <= kSmallT;  // one CTA routes and plans all pairs
@@ -456,6 +466,13 @@ moe_status moe_forward_host(const void* x_host, void* x_dev, const float* w_rout
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     return MOE_OK;
+}
+
+int32_t moe_set_combine(int32_t mode) {
+    std::lock_guard<std::mutex> lock(g_dispatch_mu);
+    const int old = g_combine;
+    if (mode == MOE_COMBINE_ATOMIC || mode == MOE_COMBINE_ORDERED) g_combine = mode;
+    return old;
 }
 
 int32_t moe_set_dispatch(int32_t mode) {

@@ -58,6 +58,22 @@ def test_workspace_bytes_and_layout(lib):
     assert lib.moe_workspace_bytes(ctypes.byref(d), 7) == 0
 
 
+def test_ordered_combine_sizes_the_slot_outputs(lib):
+    """Under the ordered combine the y_acc region holds (P, H) fp32 slot rows."""
+    d = _d(T=4096, H=2048, E=32, k=4, I=1792)
+    old = lib.moe_set_combine(abi.MOE_COMBINE_ORDERED)
+    try:
+        assert lib.moe_set_combine(abi.MOE_COMBINE_ORDERED) == abi.MOE_COMBINE_ORDERED
+        L = abi.moe_ws_layout()
+        assert lib.moe_workspace_layout(ctypes.byref(d), 0, ctypes.byref(L)) == abi.MOE_OK
+        assert L.h >= 4096 * 4 * 2048 * 4
+        ordered_total = L.total
+    finally:
+        lib.moe_set_combine(old)
+    assert lib.moe_set_combine(99) == old                     # invalid value ignored
+    assert lib.moe_workspace_bytes(ctypes.byref(d), 0) < ordered_total
+
+
 @pytest.mark.parametrize("bad,status", [
     (dict(T=-1), abi.MOE_ERR_SHAPE), (dict(H=100), abi.MOE_ERR_SHAPE), (dict(H=32), abi.MOE_ERR_SHAPE),
     (dict(I=96), abi.MOE_ERR_SHAPE), (dict(E=0), abi.MOE_ERR_SHAPE), (dict(E=257), abi.MOE_ERR_SHAPE),
