@@ -41,6 +41,17 @@ Readings where the pages are silent (each is also listed in the design doc):
   * an all-NaN row picks experts 0..k-1; its weights, and so its output row,
     are NaN;
   * relu^2 keeps NaN (u > 0 ? u : (NaN ? u : 0)) and then squares.
+
+Router and activation variants (TensorFold issue #548: the table of pieces
+each model family builds lists "routers (softmax, sigmoid + bias)"; its
+section "Paths your experts test does not reach" runs swiglu_limit 10, where
+gate and up pre-activations clamp and limit 0 is the control):
+  * score "softmax": s = exp(L - max_e L) / sum_e exp(L - max_e L) over the
+    token's E logits; the bias, if any, still only selects; a row with a NaN
+    logit scores NaN throughout;
+  * norm_topk off: w_j = s[idx_j] * scale, no division;
+  * swiglu_limit L > 0: g <- min(g, L), u <- clamp(u, -L, L) before
+    silu(g) * u, NaN kept (0 turns the clamp off).
 """
 from __future__ import annotations
 
@@ -48,7 +59,8 @@ import numpy as np
 
 __all__ = [
     "bf16_to_f64", "router_logits", "sigmoid", "select_topk", "select_topk_bruteforce",
-    "route", "tie_margins", "plan", "dequant_affine4", "silu", "swiglu", "relu2",
+    "route", "tie_margins", "plan", "dequant_affine4", "silu", "swiglu", "relu2", "softmax",
+    "clamp_swiglu_inputs",
     "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "BM",
 ]
 
@@ -77,6 +89,15 @@ def sigmoid(L: np.ndarray) -> np.ndarray:
     L = np.asarray(L, dtype=np.float64)
     with np.errstate(over="ignore", invalid="ignore"):
         return 1.0 / (1.0 + np.exp(-L))
+
+
+def softmax(L: np.ndarray) -> np.ndarray:
+    """Row-wise exp(L - max) / sum(exp(L - max)); a NaN anywhere in a row
+    makes the whole row NaN."""
+    L = np.asarray(L, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        z = np.exp(L - L.max(axis=-1, keepdims=True))
+        return z / z.sum(axis=-1, keepdims=True)
 
 
 def select_topk(c: np.ndarray, k: int) -> np.ndarray:
@@ -119,13 +140,15 @@ def select_topk_bruteforce(c_row, k: int):
 
 
 def route(*, k: int, eps: float, scale: float, expert_bias, x_bits=None, w_router=None,
-          logits=None):
-    """Sigmoid routing with a selection-only expert bias.
+          logits=None, score: str = "sigmoid", norm_topk: bool = True):
+    """Sigmoid (or softmax) routing with a selection-only expert bias.
 
     Exactly one of (x_bits with w_router) or logits (fp32, widened) is given.
     Returns a dict with L, s, c, idx (T, k) and w (T, k):
-        s = sigmoid(L);  c = s + bias (selection only);  idx = top-k of c;
-        w_j = s[idx_j] / (sum_j s[idx_j] + eps) * scale   (sum in slot order).
+        s = sigmoid(L) (or softmax(L));  c = s + bias (selection only);
+        idx = top-k of c;
+        w_j = s[idx_j] / (sum_j s[idx_j] + eps) * scale   (sum in slot order),
+        or s[idx_j] * scale with norm_topk off.
     """
     if (x_bits is None) == (logits is None):
         raise ValueError("give exactly one of x_bits or logits")
@@ -133,7 +156,12 @@ def route(*, k: int, eps: float, scale: float, expert_bias, x_bits=None, w_route
         L = router_logits(x_bits, w_router)
     else:
         L = np.asarray(logits, dtype=np.float32).astype(np.float64)
-    s = sigmoid(L)
+    if score == "sigmoid":
+        s = sigmoid(L)
+    elif score == "softmax":
+        s = softmax(L)
+    else:
+        raise ValueError(score)
     b = np.asarray(expert_bias, dtype=np.float32).astype(np.float64)
     c = s + b[None, :]
     idx = select_topk(c, k)
@@ -141,7 +169,7 @@ def route(*, k: int, eps: float, scale: float, expert_bias, x_bits=None, w_route
     tot = np.zeros(sel.shape[0])
     for j in range(k):
         tot = tot + sel[:, j]
-    w = sel / (tot + eps)[:, None] * scale
+    w = sel / (tot + eps)[:, None] * scale if norm_topk else sel * scale
     return {"L": L, "s": s, "c": c, "idx": idx, "w": w}
 
 
@@ -221,9 +249,19 @@ def _expert_w(inp, which: str, e: int) -> np.ndarray:
                            getattr(inp, which + "_bias")[e])
 
 
-def _act(h1: np.ndarray, act: str, I: int) -> np.ndarray:
+def clamp_swiglu_inputs(g, u, limit: float):
+    """g <- min(g, limit), u <- clamp(u, -limit, limit), NaN kept; limit 0
+    leaves both as they are."""
+    if not limit:
+        return g, u
+    g = np.where(g > limit, limit, g)
+    u = np.where(u > limit, limit, np.where(u < -limit, -limit, u))
+    return g, u
+
+
+def _act(h1: np.ndarray, act: str, I: int, limit: float = 0.0) -> np.ndarray:
     if act == "swiglu":
-        return swiglu(h1[:, :I], h1[:, I:2 * I])
+        return swiglu(*clamp_swiglu_inputs(h1[:, :I], h1[:, I:2 * I], limit))
     if act == "relu2":
         return relu2(h1)
     raise ValueError(act)
@@ -243,7 +281,7 @@ def expert_outputs(inp, idx: np.ndarray, tokens: np.ndarray) -> np.ndarray:
         W1 = _expert_w(inp, "w1", int(e))
         W2 = _expert_w(inp, "w2", int(e))
         with np.errstate(invalid="ignore", over="ignore"):
-            a = _act(x[rr] @ W1.T, wl.act, wl.I)
+            a = _act(x[rr] @ W1.T, wl.act, wl.I, wl.swiglu_limit)
             o[rr, jj] = a @ W2.T
     return o
 
@@ -271,10 +309,11 @@ def moe_block(inp, tokens=None, *, use_logits=None, idx=None):
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     if use_logits is not None:
         r = route(k=wl.k, eps=wl.eps, scale=wl.router_scale, expert_bias=inp.expert_bias,
-                  logits=np.asarray(use_logits)[tokens])
+                  logits=np.asarray(use_logits)[tokens], score=wl.score, norm_topk=wl.norm_topk)
     else:
         r = route(k=wl.k, eps=wl.eps, scale=wl.router_scale, expert_bias=inp.expert_bias,
-                  x_bits=inp.x_bits[tokens], w_router=inp.w_router)
+                  x_bits=inp.x_bits[tokens], w_router=inp.w_router, score=wl.score,
+                  norm_topk=wl.norm_topk)
     if idx is not None:
         idx = np.asarray(idx, dtype=np.int64)
         sel = np.take_along_axis(r["s"], idx, axis=1)
@@ -282,7 +321,7 @@ def moe_block(inp, tokens=None, *, use_logits=None, idx=None):
         for j in range(wl.k):
             tot = tot + sel[:, j]
         r["idx"] = idx
-        r["w"] = sel / (tot + wl.eps)[:, None] * wl.router_scale
+        r["w"] = sel / (tot + wl.eps)[:, None] * wl.router_scale if wl.norm_topk else sel * wl.router_scale
     o = expert_outputs(inp, r["idx"], tokens)
     acc, y = combine(o, r["w"], wl.out_scale)
     r.update({"tokens": tokens, "acc": acc, "y": y})
@@ -295,7 +334,7 @@ def moe_block_all_experts(inp):
     Tiny inputs only."""
     wl = inp.wl
     r = route(k=wl.k, eps=wl.eps, scale=wl.router_scale, expert_bias=inp.expert_bias,
-              x_bits=inp.x_bits, w_router=inp.w_router)
+              x_bits=inp.x_bits, w_router=inp.w_router, score=wl.score, norm_topk=wl.norm_topk)
     x = bf16_to_f64(inp.x_bits)
     dense_w = np.zeros((wl.T, wl.E))
     for j in range(wl.k):
@@ -303,6 +342,6 @@ def moe_block_all_experts(inp):
     acc = np.zeros((wl.T, wl.H))
     for e in range(wl.E):
         with np.errstate(invalid="ignore", over="ignore"):
-            a = _act(x @ _expert_w(inp, "w1", e).T, wl.act, wl.I)
+            a = _act(x @ _expert_w(inp, "w1", e).T, wl.act, wl.I, wl.swiglu_limit)
             acc += dense_w[:, e, None] * (a @ _expert_w(inp, "w2", e).T)
     return acc, wl.out_scale * acc

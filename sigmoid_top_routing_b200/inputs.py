@@ -56,6 +56,9 @@ class Workload:
     nan_rows: int = 0            # token rows of x set to NaN (all-NaN router logits)
     hot_experts: int = 0         # experts given a bias offset
     hot_delta: float = 0.0       # that offset (found by bisection on the oracle's routing)
+    score: str = "sigmoid"       # router score: "sigmoid" | "softmax"
+    norm_topk: bool = True       # divide the picked scores by their sum + eps
+    swiglu_limit: float = 0.0    # clamp of the SwiGLU inputs (0: off)
     seed: int = 0
 
     def with_T(self, T: int, name: Optional[str] = None) -> "Workload":

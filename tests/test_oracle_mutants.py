@@ -75,10 +75,10 @@ def test_mutant_relu2_drops_nan(monkeypatch):
 def test_mutant_gate_up_swapped(monkeypatch):
     real = OM._act
 
-    def bad(h1, act, I):
+    def bad(h1, act, I, limit=0.0):
         if act == "swiglu":
             return OM.swiglu(h1[:, I:2 * I], h1[:, :I])
-        return real(h1, act, I)
+        return real(h1, act, I, limit)
     monkeypatch.setattr(OM, "_act", bad)
     _expect_red(pins.test_one_hot_swiglu_closed_form)
 
