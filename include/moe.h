@@ -101,7 +101,12 @@ typedef struct {
  *     w1_scale, w1_bias = (E, N1, H/64) bf16;
  *     w2 = codes (E, H, I/8) uint32, w2_scale, w2_bias = (E, H, I/64) bf16.
  *     A uint32 holds 8 consecutive k, the low nibble first; the weight is
- *     scale * q + bias (TensorFold pull #1492, "What": Affine4 experts). */
+ *     scale * q + bias (TensorFold pull #1492, "What": Affine4 experts).
+ *   swiglu_limit (SWIGLU only; 0 = off, must be >= 0 and finite): before the
+ *     activation the gate is clamped from above, g = min(g, limit), and the
+ *     up value on both sides, u = clamp(u, -limit, limit); NaN stays NaN
+ *     (TensorFold issue #548, "Paths your experts test does not reach":
+ *     swiglu_limit 10, gate and up pre-activations clamp). */
 typedef struct {
     int32_t fmt; /* moe_wfmt */
     int32_t act; /* moe_act */
@@ -111,7 +116,22 @@ typedef struct {
     const void* w2;
     const void* w2_scale;
     const void* w2_bias;
+    float swiglu_limit;
 } moe_experts_w;
+
+/* Router variants (TensorFold issue #548: the pieces each model family
+ * builds include "routers (softmax, sigmoid + bias)").
+ *   score = MOE_SCORE_SIGMOID (default): s = 1 / (1 + exp(-L));
+ *           MOE_SCORE_SOFTMAX: s = exp(L - max L) / sum exp(L - max L) over
+ *           the token's E logits (a NaN logit makes the row's scores NaN).
+ *   The expert bias is added to s for selection only, either way.
+ *   norm_topk = 1 (default): w_j = s_j / (sum of the k picked s + eps) * scale;
+ *             = 0:           w_j = s_j * scale. */
+typedef enum { MOE_SCORE_SIGMOID = 0, MOE_SCORE_SOFTMAX = 1 } moe_score;
+typedef struct {
+    int32_t score;     /* moe_score */
+    int32_t norm_topk; /* 0 or 1 */
+} moe_router_cfg;
 
 /* The routing plan (device arrays the caller allocates).
  *   counts  [E]    pairs routed to each expert
@@ -178,6 +198,21 @@ MOE_API moe_status moe_forward(const void* x, const float* logits, const float* 
                        float out_scale, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
                        const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream);
+
+/* moe_route and moe_forward with a router configuration (NULL = the
+ * defaults above: sigmoid scores, normalised top-k).  Everything else as
+ * moe_route / moe_forward; MOE_ERR_UNSUPPORTED for an unknown score or a
+ * norm_topk other than 0 or 1. */
+MOE_API moe_status moe_route_ex(const void* x, const float* logits, const float* w_router,
+                                const float* expert_bias, const moe_dims* d, float eps, float scale,
+                                const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w,
+                                moe_stream_t stream);
+MOE_API moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
+                                  const float* expert_bias, const moe_dims* d, float eps,
+                                  float router_scale, float out_scale, const moe_router_cfg* cfg,
+                                  const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
+                                  const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
+                                  moe_stream_t stream);
 
 /* moe_forward with HOST buffers for the token rows: x_host (T, H) bf16 is
  * copied to x_dev, the block runs, and y_dev is copied back to y_host (T, H)

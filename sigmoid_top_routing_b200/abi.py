@@ -21,6 +21,7 @@ MOE_ACT_SWIGLU, MOE_ACT_RELU2 = 0, 1
 MOE_W_BF16, MOE_W_AFFINE4_G64 = 0, 1
 MOE_DISPATCH_AUTO, MOE_DISPATCH_GEMV, MOE_DISPATCH_GEMM = 0, 1, 2
 MOE_COMBINE_ATOMIC, MOE_COMBINE_ORDERED = 0, 1
+MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX = 0, 1
 MOE_STAGE_ROUTE, MOE_STAGE_PLAN, MOE_STAGE_UP, MOE_STAGE_DOWN, MOE_STAGE_FINAL, MOE_STAGE_GATHER = range(6)
 MOE_TILE_M = 128
 
@@ -32,7 +33,12 @@ class moe_dims(ctypes.Structure):
 class moe_experts_w(ctypes.Structure):
     _fields_ = [("fmt", c_int32), ("act", c_int32),
                 ("w1", c_void_p), ("w1_scale", c_void_p), ("w1_bias", c_void_p),
-                ("w2", c_void_p), ("w2_scale", c_void_p), ("w2_bias", c_void_p)]
+                ("w2", c_void_p), ("w2_scale", c_void_p), ("w2_bias", c_void_p),
+                ("swiglu_limit", c_float)]
+
+
+class moe_router_cfg(ctypes.Structure):
+    _fields_ = [("score", c_int32), ("norm_topk", c_int32)]
 
 
 class moe_plan_t(ctypes.Structure):
@@ -57,6 +63,11 @@ PROTOTYPES = {
     "moe_forward": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
                               c_float, POINTER(moe_experts_w), c_void_p, c_void_p, POINTER(moe_plan_t),
                               c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_route_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
+                               POINTER(moe_router_cfg), c_void_p, c_void_p, c_void_p]),
+    "moe_forward_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
+                                 c_float, POINTER(moe_router_cfg), POINTER(moe_experts_w), c_void_p, c_void_p,
+                                 POINTER(moe_plan_t), c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_host": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float,
                                    c_float, c_float, POINTER(moe_experts_w), c_void_p, c_void_p,
                                    POINTER(moe_plan_t), c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -54,10 +54,16 @@ class ExpertWeights:
     w1_bias: Optional[torch.Tensor] = None
     w2_scale: Optional[torch.Tensor] = None
     w2_bias: Optional[torch.Tensor] = None
+    swiglu_limit: float = 0.0
 
     def c_struct(self) -> abi.moe_experts_w:
         return abi.moe_experts_w(self.fmt, self.act, _ptr(self.w1), _ptr(self.w1_scale), _ptr(self.w1_bias),
-                                 _ptr(self.w2), _ptr(self.w2_scale), _ptr(self.w2_bias))
+                                 _ptr(self.w2), _ptr(self.w2_scale), _ptr(self.w2_bias), self.swiglu_limit)
+
+
+def router_cfg(score: str = "sigmoid", norm_topk: bool = True) -> abi.moe_router_cfg:
+    return abi.moe_router_cfg({"sigmoid": abi.MOE_SCORE_SIGMOID, "softmax": abi.MOE_SCORE_SOFTMAX}[score],
+                              1 if norm_topk else 0)
 
 
 @dataclasses.dataclass
@@ -97,7 +103,8 @@ def new_workspace(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16, device="cuda") -> 
 
 
 def moe_route(x=None, logits=None, w_router=None, expert_bias=None, *, E: int, k: int, eps: float = 1e-6,
-              scale: float = 1.0, topk_idx=None, topk_w=None, stream=None):
+              scale: float = 1.0, topk_idx=None, topk_w=None, stream=None, score: str = "sigmoid",
+              norm_topk: bool = True):
     src = x if x is not None else logits
     T = src.shape[0]
     H = x.shape[1] if x is not None else (w_router.shape[1] if w_router is not None else 64)
@@ -107,8 +114,10 @@ def moe_route(x=None, logits=None, w_router=None, expert_bias=None, *, E: int, k
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=dev)
-    check(load().moe_route(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d),
-                           eps, scale, _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    rc = router_cfg(score, norm_topk)
+    check(load().moe_route_ex(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d),
+                              eps, scale, ctypes.byref(rc), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+          "moe_route")
     return topk_idx, topk_w
 
 
@@ -139,7 +148,8 @@ def moe_experts(x, plan: Plan, topk_w, W: ExpertWeights, *, E: int, I: int, out_
 
 def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int, k: int, I: int,
                 logits=None, eps: float = 1e-6, router_scale: float = 1.0, out_scale: float = 1.0,
-                topk_idx=None, topk_w=None, plan: Optional[Plan] = None, y=None, ws=None, stream=None):
+                topk_idx=None, topk_w=None, plan: Optional[Plan] = None, y=None, ws=None, stream=None,
+                score: str = "sigmoid", norm_topk: bool = True):
     T, H = x.shape
     d = abi.moe_dims(T, H, E, k, I)
     dev = x.device
@@ -148,10 +158,11 @@ def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int,
     plan = plan or new_plan(T, E, k, dev)
     y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     ws = ws if ws is not None else new_workspace(d, W.fmt, dev)
-    cp, cw = plan.c_struct(), W.c_struct()
-    check(load().moe_forward(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d), eps,
-                             router_scale, out_scale, ctypes.byref(cw), _ptr(topk_idx), _ptr(topk_w),
-                             ctypes.byref(cp), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "moe_forward")
+    cp, cw, rc = plan.c_struct(), W.c_struct(), router_cfg(score, norm_topk)
+    check(load().moe_forward_ex(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d), eps,
+                                router_scale, out_scale, ctypes.byref(rc), ctypes.byref(cw), _ptr(topk_idx),
+                                _ptr(topk_w), ctypes.byref(cp), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
+          "moe_forward")
     return y, topk_idx, topk_w, plan
 
 

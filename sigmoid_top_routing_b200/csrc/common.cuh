@@ -79,6 +79,15 @@ MOE_DEV float warp_sum(float v) {
 // SwiGLU and relu^2 activations in fp32.
 // silu(g) * u with the logistic computed as 1 / (1 + exp(-g)).
 MOE_DEV float act_swiglu(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+// The SwiGLU input clamp (limit > 0): gate from above, up on both sides;
+// comparisons keep NaN (NaN > L is false).
+MOE_DEV void clamp_swiglu(float& g, float& u, float limit) {
+    if (limit > 0.0f) {
+        g = g > limit ? limit : g;
+        u = u > limit ? limit : (u < -limit ? -limit : u);
+    }
+}
 // relu(u)^2 that keeps NaN: a NaN input is squared (stays NaN), never clamped.
 MOE_DEV float act_relu2(float u) {
     float r = (u > 0.0f || u != u) ? u : 0.0f;

@@ -92,6 +92,8 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
     if (W->act != MOE_ACT_SWIGLU && W->act != MOE_ACT_RELU2)
         return fail(MOE_ERR_UNSUPPORTED, "unknown activation");
     if (!aligned16(W->w1) || !aligned16(W->w2)) return fail(MOE_ERR_ALIGN, "w1/w2 not 16-byte aligned");
+    if (!(W->swiglu_limit >= 0.0f) || W->swiglu_limit > 3.0e38f)
+        return fail(MOE_ERR_SHAPE, "swiglu_limit must be finite and >= 0 (0 = off)");
 
     // scratch layout: y_acc fp32 (T, H) | h bf16 (P, I) | router-logit scratch
     const size_t T = d->T, H = d->H, I = d->I, E = d->E, P = T * d->k;
@@ -171,6 +173,7 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
     a.I = d->I;
     a.act = W->act;
     a.fmt = W->fmt;
+    a.swiglu_limit = W->swiglu_limit;
     a.w1 = W->w1;
     a.w2 = W->w2;
     a.h = h;

@@ -66,6 +66,7 @@ struct GemmParams {
     int feats;               // output features per expert: I (up) or H (down)
     const uint16_t* wscale;  // affine 4-bit: (E, rows_per_expert, K/64) bf16 scales
     const uint16_t* wbias;   //                and biases
+    float swiglu_limit;      // up SwiGLU: clamp of the gate (above) and up (both sides); 0 off
     int* err;
 };
 
@@ -584,7 +585,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
-                            if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(v[i], u[i]));
+                            if (c >= tl.ntok) continue;
+                            float gv = v[i], uv = u[i];
+                            clamp_swiglu(gv, uv, g.swiglu_limit);
+                            g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(gv, uv));
                         }
                     }
                 } else {
@@ -599,8 +603,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
-                            if (c < tl.ntok)
-                                g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(v[i], s_u[lrow * 17 + i]));
+                            if (c >= tl.ntok) continue;
+                            float gv = v[i], uv = s_u[lrow * 17 + i];
+                            clamp_swiglu(gv, uv, g.swiglu_limit);
+                            g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(gv, uv));
                         }
                     }
                     named_bar(1, 128);
@@ -724,6 +730,7 @@ GemmParams params(const ExpertArgs& a, bool up) {
         g.feats = a.I;
         g.wscale = a.w1_scale;
         g.wbias = a.w1_bias;
+        g.swiglu_limit = a.swiglu_limit;
     } else {
         g.K = a.I;
         g.rows_per_expert = a.H;

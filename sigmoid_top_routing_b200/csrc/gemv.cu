@@ -124,7 +124,9 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_gemv_up(ExpertArgs a) {
 #pragma unroll
             for (int m = 0; m < kTokGroup; ++m) {
                 if (m < mt && lane == m) {
-                    const float v = ACT == 0 ? act_swiglu(sg[m], su[m]) : act_relu2(sg[m]);
+                    float gv = sg[m], uv = su[m];
+                    if (ACT == 0) clamp_swiglu(gv, uv, a.swiglu_limit);
+                    const float v = ACT == 0 ? act_swiglu(gv, uv) : act_relu2(gv);
                     a.h[(size_t)(off + m0 + m) * I + r] = f2bf16(v);
                 }
             }

@@ -234,7 +234,9 @@ __global__ void __launch_bounds__(kA4Warps * 32, 4) k_gemv_a4(ExpertArgs a) {
                 if (n >= nt) continue;
                 const int slot = slot0 + n;
                 if (MODE == kA4UpSwiglu) {
-                    a.h[(size_t)slot * a.I + rb * 8 + g] = f2bf16(act_swiglu(acc[jn], acc[2 + jn]));
+                    float gv = acc[jn], uv = acc[2 + jn];
+                    clamp_swiglu(gv, uv, a.swiglu_limit);
+                    a.h[(size_t)slot * a.I + rb * 8 + g] = f2bf16(act_swiglu(gv, uv));
                 } else if (MODE == kA4UpRelu2) {
                     a.h[(size_t)slot * a.I + rb * 16 + g] = f2bf16(act_relu2(acc[jn]));
                     a.h[(size_t)slot * a.I + rb * 16 + g + 8] = f2bf16(act_relu2(acc[2 + jn]));

@@ -17,6 +17,8 @@ struct RouteArgs {
     float* part;             // (8, T, E) fp32 per-segment partial logits, or null
     int T, H, E, k;
     float eps, scale;
+    int softmax;             // 1: softmax scores over the E logits; 0: sigmoid
+    int no_norm;             // 1: w = s * scale (no division by the picked sum)
     int32_t* idx;            // (T, k)
     float* w;                // (T, k)
     // optional fused plan (single-CTA select path only)
@@ -46,6 +48,7 @@ struct ExpertArgs {
     int T, H, E, k, I;
     int act;                 // 0 swiglu, 1 relu2
     int fmt;                 // 0 bf16, 1 affine4
+    float swiglu_limit;      // > 0: g = min(g, L), u = clamp(u, -L, L) before silu(g) * u
     const void* w1;
     const uint16_t* w1_scale;
     const uint16_t* w1_bias;

@@ -157,6 +157,19 @@ moe_status check_weights(const moe_experts_w* W) {
             !aligned16(W->w2_bias))
             return fail(MOE_ERR_ALIGN, "affine-4 scale/bias not 16-byte aligned");
     }
+    if (!(W->swiglu_limit >= 0.0f) || W->swiglu_limit > 3.0e38f)
+        return fail(MOE_ERR_SHAPE, "swiglu_limit must be finite and >= 0 (0 = off)");
+    return MOE_OK;
+}
+
+// The router configuration (NULL: sigmoid scores, normalised top-k).
+moe_status check_router_cfg(const moe_router_cfg* cfg, RouteArgs* r) {
+    if (!cfg) return MOE_OK;
+    if (cfg->score != MOE_SCORE_SIGMOID && cfg->score != MOE_SCORE_SOFTMAX)
+        return fail(MOE_ERR_UNSUPPORTED, "router score %d", cfg->score);
+    if (cfg->norm_topk != 0 && cfg->norm_topk != 1) return fail(MOE_ERR_UNSUPPORTED, "norm_topk %d", cfg->norm_topk);
+    r->softmax = cfg->score == MOE_SCORE_SOFTMAX;
+    r->no_norm = cfg->norm_topk == 0;
     return MOE_OK;
 }
 
@@ -206,6 +219,7 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.I = d->I;
     a.act = W->act;
     a.fmt = W->fmt;
+    a.swiglu_limit = W->swiglu_limit;
     a.w1 = W->w1;
     a.w1_scale = static_cast<const uint16_t*>(W->w1_scale);
     a.w1_bias = static_cast<const uint16_t*>(W->w1_bias);
@@ -323,11 +337,18 @@ moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* o
 moe_status moe_route(const void* x, const float* logits, const float* w_router,
                      const float* expert_bias, const moe_dims* d, float eps, float scale,
                      int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+    return moe_route_ex(x, logits, w_router, expert_bias, d, eps, scale, nullptr, topk_idx, topk_w, stream);
+}
+
+moe_status moe_route_ex(const void* x, const float* logits, const float* w_router,
+                        const float* expert_bias, const moe_dims* d, float eps, float scale,
+                        const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    RouteArgs a{};
+    if ((st = check_router_cfg(cfg, &a)) != MOE_OK) return st;
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
     if ((st = check_route_args(x, logits, w_router, d, topk_idx, topk_w)) != MOE_OK) return st;
-    RouteArgs a{};
     a.x = static_cast<const uint16_t*>(x);
     a.logits = logits;
     a.w_router = w_router;
@@ -394,8 +415,19 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
                        float out_scale, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
                        const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
+    return moe_forward_ex(x, logits, w_router, expert_bias, d, eps, router_scale, out_scale, nullptr, W,
+                          topk_idx, topk_w, plan, y, ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
+                          const float* expert_bias, const moe_dims* d, float eps, float router_scale,
+                          float out_scale, const moe_router_cfg* cfg, const moe_experts_w* W,
+                          int32_t* topk_idx, float* topk_w, const moe_plan_t* plan, void* y, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    RouteArgs r0{};
+    if ((st = check_router_cfg(cfg, &r0)) != MOE_OK) return st;
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
     if (!x || !y) return fail(MOE_ERR_NULL, "x or y is NULL (both are needed by the experts)");
     if (!aligned16(x) || !aligned16(y)) return fail(MOE_ERR_ALIGN, "x or y not 16-byte aligned");
@@ -420,6 +452,8 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
     r.k = d->k;
     r.eps = eps;
     r.scale = router_scale;
+    r.softmax = r0.softmax;
+    r.no_norm = r0.no_norm;
     r.idx = topk_idx;
     r.w = topk_w;
     r.counts = plan->counts;

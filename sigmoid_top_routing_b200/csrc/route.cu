@@ -43,15 +43,43 @@ MOE_DEV float sigmoid_f32(float L) { return 1.0f / (1.0f + expf(-L)); }
 // Lane j (< k) returns slot j's expert in *e_out (and writes idx/w rows).
 template <int NE>
 MOE_DEV int select_token(const float (&Lv)[NE], const float* __restrict__ bias, int E, int k,
-                         float eps, float scale, int32_t* idx_row, float* w_row) {
+                         float eps, float scale, bool softmax, bool no_norm, int32_t* idx_row,
+                         float* w_row) {
     const int lane = threadIdx.x & 31;
     float s[NE];
     uint32_t khi[NE], klo[NE];
+    // softmax: exp(L - max) / sum over the row (warp reductions); a NaN logit
+    // makes every score of the row NaN
+    float smax = 0.0f, sinv = 0.0f;
+    bool row_nan = false;
+    if (softmax) {
+        float m = -INFINITY;
+        bool nan_here = false;
+#pragma unroll
+        for (int i = 0; i < NE; ++i) {
+            if (lane + 32 * i < E) {
+                if (Lv[i] != Lv[i]) nan_here = true;
+                else m = fmaxf(m, Lv[i]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        row_nan = __any_sync(0xffffffffu, nan_here);
+        float z = 0.0f;
+#pragma unroll
+        for (int i = 0; i < NE; ++i)
+            if (lane + 32 * i < E) z += expf(Lv[i] - m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+        smax = m;
+        sinv = z;
+    }
 #pragma unroll
     for (int i = 0; i < NE; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
-            s[i] = sigmoid_f32(Lv[i]);
+            s[i] = softmax ? (row_nan ? __int_as_float(0x7fc00000) : expf(Lv[i] - smax) / sinv)
+                           : sigmoid_f32(Lv[i]);
             const float c = s[i] + (bias ? __ldg(bias + e) : 0.0f);
             khi[i] = score_key(c);
             klo[i] = 0xFFFFFFFFu - (uint32_t)e;
@@ -92,7 +120,7 @@ MOE_DEV int select_token(const float (&Lv)[NE], const float* __restrict__ bias, 
     const float denom = sum + eps;
     if (lane < k) {
         idx_row[lane] = my_e;
-        w_row[lane] = my_s / denom * scale;
+        w_row[lane] = no_norm ? my_s * scale : my_s / denom * scale;
     }
     return my_e;
 }
@@ -181,8 +209,8 @@ __global__ void __launch_bounds__(256) k_select(RouteArgs a) {
                 Lv[i] = e < a.E ? L[(size_t)t * a.E + e] : 0.0f;
             }
         }
-        const int e = select_token<NE>(Lv, a.bias, a.E, a.k, a.eps, a.scale, a.idx + (size_t)t * a.k,
-                                       a.w + (size_t)t * a.k);
+        const int e = select_token<NE>(Lv, a.bias, a.E, a.k, a.eps, a.scale, a.softmax != 0, a.no_norm != 0,
+                                       a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k);
         if (FUSE && lane < a.k) s_idx[t * a.k + lane] = e;
     }
     if (FUSE) {
@@ -344,8 +372,8 @@ __global__ void __launch_bounds__(256) k_route_large(RouteArgs a) {
             for (int w = 1; w < kSegs; ++w) L += part[(w * TT + m) * EP + e];
             Lv[i] = L;
         }
-        select_token<NE>(Lv, a.bias, E, a.k, a.eps, a.scale, a.idx + (size_t)t * a.k,
-                         a.w + (size_t)t * a.k);
+        select_token<NE>(Lv, a.bias, E, a.k, a.eps, a.scale, a.softmax != 0, a.no_norm != 0,
+                         a.idx + (size_t)t * a.k, a.w + (size_t)t * a.k);
     }
     pdl_trigger();
 }

@@ -35,12 +35,13 @@ def to_device(inp: MoEInputs, device="cuda", with_x: bool = True) -> DeviceInput
     act = abi.MOE_ACT_SWIGLU if wl.act == "swiglu" else abi.MOE_ACT_RELU2
     if wl.fmt == "bf16":
         W = ExpertWeights(act=act, fmt=abi.MOE_W_BF16, w1=bf16_tensor(inp.w1_bits, device),
-                          w2=bf16_tensor(inp.w2_bits, device))
+                          w2=bf16_tensor(inp.w2_bits, device), swiglu_limit=wl.swiglu_limit)
     else:
         W = ExpertWeights(act=act, fmt=abi.MOE_W_AFFINE4_G64,
                           w1=u32_tensor(inp.w1_q, device), w2=u32_tensor(inp.w2_q, device),
                           w1_scale=bf16_tensor(inp.w1_scale, device), w1_bias=bf16_tensor(inp.w1_bias, device),
-                          w2_scale=bf16_tensor(inp.w2_scale, device), w2_bias=bf16_tensor(inp.w2_bias, device))
+                          w2_scale=bf16_tensor(inp.w2_scale, device), w2_bias=bf16_tensor(inp.w2_bias, device),
+                          swiglu_limit=wl.swiglu_limit)
     x = bf16_tensor(inp.x_bits, device) if with_x else None
     return DeviceInputs(x=x, w_router=torch.from_numpy(inp.w_router).to(device),
                         expert_bias=torch.from_numpy(inp.expert_bias).to(device), W=W)

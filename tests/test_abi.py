@@ -138,6 +138,27 @@ def test_experts_refuses_bad_weights(lib):
     assert call(_weights(), y=None) == abi.MOE_ERR_NULL
 
 
+def test_swiglu_limit_must_be_finite_and_non_negative(lib):
+    d = _d()
+    n = lib.moe_workspace_bytes(ctypes.byref(d), 0)
+    p = _plan()
+    for bad in (-1.0, float("nan"), float("inf")):
+        W = _weights()
+        W.swiglu_limit = bad
+        assert lib.moe_experts(0x10000, ctypes.byref(p), 0x30000, ctypes.byref(d), ctypes.byref(W), 1.0,
+                               0x20000, 0x1000000, n, None) == abi.MOE_ERR_SHAPE
+
+
+def test_router_cfg_refuses_unknown_modes(lib):
+    d = _d()
+    for cfg in (abi.moe_router_cfg(7, 1), abi.moe_router_cfg(0, 2)):
+        assert lib.moe_route_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, ctypes.byref(cfg),
+                                0x30000, 0x40000, None) == abi.MOE_ERR_UNSUPPORTED
+        assert lib.moe_forward_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, 1.0,
+                                  ctypes.byref(cfg), ctypes.byref(_weights()), 0x30000, 0x40000,
+                                  ctypes.byref(_plan()), 0x50000, 0x1000000, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+
+
 def test_forward_refuses_missing_router(lib):
     d = _d()
     n = lib.moe_workspace_bytes(ctypes.byref(d), 0)

@@ -51,7 +51,7 @@ def run_forward(api, inp, *, dispatch=None, logits=None, poison=True):
         lg = None if logits is None else torch.from_numpy(logits).cuda()
         api.moe_forward(D.x, D.W, D.w_router, D.expert_bias, E=wl.E, k=wl.k, I=wl.I, logits=lg,
                         eps=wl.eps, router_scale=wl.router_scale, out_scale=wl.out_scale, topk_idx=idx,
-                        topk_w=w, plan=plan, y=y, ws=ws)
+                        topk_w=w, plan=plan, y=y, ws=ws, score=wl.score, norm_topk=wl.norm_topk)
         torch.cuda.synchronize()
         assert api.moe_device_error() == 0
     finally:
