@@ -52,6 +52,12 @@ gate and up pre-activations clamp and limit 0 is the control):
   * norm_topk off: w_j = s[idx_j] * scale, no division;
   * swiglu_limit L > 0: g <- min(g, L), u <- clamp(u, -L, L) before
     silu(g) * u, NaN kept (0 turns the clamp off).
+
+Shared expert (vllm.cpp PR #684, "The finding that justifies the row": the
+combine multiplies the routed sum by the routed scale BEFORE the shared
+expert's output is added; the shared output itself is not scaled):
+    y = out_scale * sum_j w_j * o_j  +  down_s(act(up_s(x)))
+with the shared expert's own width I_s, the block's activation, weight 1.
 """
 from __future__ import annotations
 
@@ -61,7 +67,7 @@ __all__ = [
     "bf16_to_f64", "router_logits", "sigmoid", "select_topk", "select_topk_bruteforce",
     "route", "tie_margins", "plan", "dequant_affine4", "silu", "swiglu", "relu2", "softmax",
     "clamp_swiglu_inputs",
-    "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "BM",
+    "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "shared_expert", "BM",
 ]
 
 BM = 128  # rows of one GEMM M-tile; the plan's tile table counts ceil(count / BM) per expert
@@ -286,6 +292,24 @@ def expert_outputs(inp, idx: np.ndarray, tokens: np.ndarray) -> np.ndarray:
     return o
 
 
+def _shared_w(inp, which: str) -> np.ndarray:
+    """float64 (N, K) weight of the shared expert."""
+    sh = inp.shared
+    if inp.wl.fmt == "bf16":
+        return bf16_to_f64(sh[which + "_bits"][0])
+    return dequant_affine4(sh[which + "_q"][0], sh[which + "_scale"][0], sh[which + "_bias"][0])
+
+
+def shared_expert(inp, tokens: np.ndarray) -> np.ndarray:
+    """sh[r] = down_s(act(up_s(x_t))) for t = tokens[r]: the shared expert,
+    on every token, with weight 1."""
+    wl = inp.wl
+    x = bf16_to_f64(inp.x_bits[tokens])
+    with np.errstate(invalid="ignore", over="ignore"):
+        a = _act(x @ _shared_w(inp, "w1").T, wl.act, wl.shared_I, wl.swiglu_limit)
+        return a @ _shared_w(inp, "w2").T
+
+
 def combine(o: np.ndarray, w: np.ndarray, out_scale: float, dtype=np.float64):
     """acc = sum_j w_j * o_j in slot order, then y = out_scale * acc: one
     multiply on the finished sum (vllm.cpp PR #684).  ``dtype`` float32 gives
@@ -324,6 +348,10 @@ def moe_block(inp, tokens=None, *, use_logits=None, idx=None):
         r["w"] = sel / (tot + wl.eps)[:, None] * wl.router_scale if wl.norm_topk else sel * wl.router_scale
     o = expert_outputs(inp, r["idx"], tokens)
     acc, y = combine(o, r["w"], wl.out_scale)
+    if wl.shared_I:
+        sh = shared_expert(inp, tokens)
+        y = y + sh                                   # after the routed scale, unscaled
+        r["shared"] = sh
     r.update({"tokens": tokens, "acc": acc, "y": y})
     return r
 

@@ -59,6 +59,7 @@ class Workload:
     score: str = "sigmoid"       # router score: "sigmoid" | "softmax"
     norm_topk: bool = True       # divide the picked scores by their sum + eps
     swiglu_limit: float = 0.0    # clamp of the SwiGLU inputs (0: off)
+    shared_I: int = 0            # intermediate width of a shared expert (0: none)
     seed: int = 0
 
     def with_T(self, T: int, name: Optional[str] = None) -> "Workload":
@@ -161,6 +162,10 @@ class MoEInputs:
     w2_bias: Optional[np.ndarray] = None
     nan_rows: Optional[np.ndarray] = None
     hot: Optional[np.ndarray] = None
+    # shared expert (one expert, same format and activation, width shared_I):
+    # keys w1_bits, w2_bits (bf16) or w1_q, w1_scale, w1_bias, w2_q, ... (affine),
+    # each with a leading dimension of 1
+    shared: Optional[dict] = None
 
     @property
     def n1(self) -> int:
@@ -194,8 +199,8 @@ def make_inputs(wl: Workload, *, with_experts: bool = True, hot_delta: Optional[
 
     ``with_experts=False`` skips the expert weights (router-only studies);
     ``hot_delta`` overrides the recorded hot-expert offset."""
-    ss = np.random.SeedSequence(wl.seed).spawn(6)
-    r_x, r_wr, r_b, r_w1, r_w2, r_extra = (np.random.default_rng(s) for s in ss)
+    ss = np.random.SeedSequence(wl.seed).spawn(7)     # the first six streams do not depend on the count
+    r_x, r_wr, r_b, r_w1, r_w2, r_extra, r_shared = (np.random.default_rng(s) for s in ss)
     T, H, E, I = wl.T, wl.H, wl.E, wl.I
     x = _normal_f32(r_x, (T, H), 1.0)
     w_router = _normal_f32(r_wr, (E, H), 0.02)
@@ -216,6 +221,13 @@ def make_inputs(wl: Workload, *, with_experts: bool = True, hot_delta: Optional[
     if with_experts:
         w1, q1, s1, b1 = _expert_weights(r_w1, E, n1, H, wl.fmt)
         w2, q2, s2, b2 = _expert_weights(r_w2, E, H, I, wl.fmt)
+    shared = None
+    if with_experts and wl.shared_I:
+        Is = wl.shared_I
+        sw1, sq1, ss1, sb1 = _expert_weights(r_shared, 1, (2 if wl.act == "swiglu" else 1) * Is, H, wl.fmt)
+        sw2, sq2, ss2, sb2 = _expert_weights(r_shared, 1, H, Is, wl.fmt)
+        shared = {"w1_bits": sw1, "w2_bits": sw2, "w1_q": sq1, "w1_scale": ss1, "w1_bias": sb1,
+                  "w2_q": sq2, "w2_scale": ss2, "w2_bias": sb2}
     return MoEInputs(wl=wl, x_bits=f32_to_bf16_bits(x), w_router=w_router, expert_bias=bias,
                      w1_bits=w1, w2_bits=w2, w1_q=q1, w1_scale=s1, w1_bias=b1,
-                     w2_q=q2, w2_scale=s2, w2_bias=b2, nan_rows=nan_rows, hot=hot)
+                     w2_q=q2, w2_scale=s2, w2_bias=b2, nan_rows=nan_rows, hot=hot, shared=shared)

@@ -148,3 +148,64 @@ def test_mutant_norm_flag_ignored(monkeypatch):
         return real(**kw)
     monkeypatch.setattr(oracle, "route", bad)
     _expect_red(test_norm_topk_off_keeps_the_raw_scores, "sigmoid")
+
+
+# ------------------------------------------------------------------ shared expert
+
+def _with_shared(inp, sw1, sw2, shared_I, **wl_over):
+    wl = dataclasses.replace(inp.wl, shared_I=shared_I, **wl_over)
+    import sigmoid_top_routing_b200.inputs as G
+    return dataclasses.replace(inp, wl=wl, shared={"w1_bits": G.f32_to_bf16_bits(sw1[None]),
+                                                   "w2_bits": G.f32_to_bf16_bits(sw2[None])})
+
+
+def test_shared_expert_one_hot_closed_form():
+    """Routed experts zeroed (their outputs are exactly 0); the shared expert of
+    width 12 holds g / u at column h0 and shifts activation i to output i + 1:
+    y[t, (i + 1) % 12] = silu(g_i) * u_i, whatever the routing."""
+    inp, _, _ = pins._one_hot_inputs("swiglu")
+    inp = dataclasses.replace(inp, w1_bits=np.zeros_like(inp.w1_bits))
+    Is, H = 12, inp.wl.H
+    g = np.arange(-3.0, 3.0, 0.5).astype(np.float32)          # exact in bf16
+    u = np.arange(2.0, -1.0, -0.25).astype(np.float32)
+    sw1 = np.zeros((2 * Is, H), np.float32)
+    sw1[:Is, 5] = g                                   # x = e_5 in the one-hot inputs
+    sw1[Is:, 5] = u
+    sw2 = np.zeros((H, Is), np.float32)
+    sw2[:Is, :] = np.roll(np.eye(Is, dtype=np.float32), 1, axis=0)
+    inp = _with_shared(inp, sw1, sw2, Is, out_scale=2.5)
+    r = oracle.moe_block(inp)
+    gd = g.astype(np.float64)
+    want = np.zeros(H)
+    want[:Is] = np.roll(gd * scipy.special.expit(gd) * u, 1)
+    for t in range(inp.wl.T):
+        np.testing.assert_allclose(r["y"][t], want, rtol=1e-13, atol=1e-15)
+
+
+def test_shared_term_is_added_after_the_routed_scale():
+    """y = out_scale * acc + sh with sh computed here by an explicit loop over
+    rows (relu^2, width 40); the shared term itself is not scaled."""
+    import sigmoid_top_routing_b200.inputs as G
+    wl = G.Workload("sh", T=6, H=64, E=4, k=2, I=32, act="relu2", out_scale=2.5)
+    inp = G.make_inputs(wl)
+    rng = _rng(9)
+    Is = 40
+    sw1 = (rng.standard_normal((Is, 64)) * 0.1).astype(np.float32)
+    sw2 = (rng.standard_normal((64, Is)) * 0.1).astype(np.float32)
+    inp = _with_shared(inp, sw1, sw2, Is)
+    r = oracle.moe_block(inp)
+    x = oracle.bf16_to_f64(inp.x_bits)
+    W1 = oracle.bf16_to_f64(inp.shared["w1_bits"][0])
+    W2 = oracle.bf16_to_f64(inp.shared["w2_bits"][0])
+    for t in range(wl.T):
+        hmid = [sum(W1[i, h] * x[t, h] for h in range(64)) for i in range(Is)]
+        a = [max(v, 0.0) ** 2 for v in hmid]
+        sh = np.array([sum(W2[n, i] * a[i] for i in range(Is)) for n in range(64)])
+        np.testing.assert_allclose(r["y"][t], 2.5 * r["acc"][t] + sh, rtol=1e-12, atol=1e-14)
+        assert not np.allclose(r["y"][t], 2.5 * (r["acc"][t] + sh), rtol=1e-6)
+
+
+def test_mutant_shared_term_scaled_too(monkeypatch):
+    real = OM.shared_expert
+    monkeypatch.setattr(OM, "shared_expert", lambda inp, tokens: inp.wl.out_scale * real(inp, tokens))
+    _expect_red(test_shared_term_is_added_after_the_routed_scale)
