@@ -202,7 +202,11 @@ MOE_API moe_status moe_forward(const void* x, const float* logits, const float* 
 /* moe_route and moe_forward with a router configuration (NULL = the
  * defaults above: sigmoid scores, normalised top-k).  Everything else as
  * moe_route / moe_forward; MOE_ERR_UNSUPPORTED for an unknown score or a
- * norm_topk other than 0 or 1. */
+ * norm_topk other than 0 or 1.  moe_forward_ex also takes y_shared, an fp32
+ * (T, H) shared-expert output (from moe_shared_expert) or NULL: the output is
+ * then y = bf16_rn(out_scale * routed sum + y_shared) -- the routed scale
+ * multiplies the routed sum before the shared term is added, which itself is
+ * not scaled (vllm.cpp PR #684, "The finding that justifies the row"). */
 MOE_API moe_status moe_route_ex(const void* x, const float* logits, const float* w_router,
                                 const float* expert_bias, const moe_dims* d, float eps, float scale,
                                 const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w,
@@ -210,9 +214,21 @@ MOE_API moe_status moe_route_ex(const void* x, const float* logits, const float*
 MOE_API moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
                                   const float* expert_bias, const moe_dims* d, float eps,
                                   float router_scale, float out_scale, const moe_router_cfg* cfg,
-                                  const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
+                                  const float* y_shared, const moe_experts_w* W, int32_t* topk_idx,
+                                  float* topk_w,
                                   const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
                                   moe_stream_t stream);
+
+/* The shared expert: one expert applied to every token with weight 1,
+ *   y_shared[t] = down_s(act(up_s(x[t])))   (fp32 (T, H), overwritten),
+ * for moe_forward_ex's y_shared.  d = {T, H, E = 1, k = 1, I = the shared
+ * expert's width}; Ws has the same layout as one expert of moe_experts_w
+ * (E = 1; act, fmt and swiglu_limit as for the routed experts).  The
+ * workspace is moe_workspace_bytes(d, Ws->fmt) for that d.  Runs the same
+ * kernels as the routed experts (tcgen05 GEMM or GEMV, per moe_set_dispatch)
+ * over a one-expert identity plan.  MOE_ERR_SHAPE unless E == 1 and k == 1. */
+MOE_API moe_status moe_shared_expert(const void* x, const moe_experts_w* Ws, const moe_dims* d,
+                                     float* y_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_forward with HOST buffers for the token rows: x_host (T, H) bf16 is
  * copied to x_dev, the block runs, and y_dev is copied back to y_host (T, H)

@@ -66,8 +66,10 @@ PROTOTYPES = {
     "moe_route_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
                                POINTER(moe_router_cfg), c_void_p, c_void_p, c_void_p]),
     "moe_forward_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
-                                 c_float, POINTER(moe_router_cfg), POINTER(moe_experts_w), c_void_p, c_void_p,
-                                 POINTER(moe_plan_t), c_void_p, c_void_p, c_size_t, c_void_p]),
+                                 c_float, POINTER(moe_router_cfg), c_void_p, POINTER(moe_experts_w), c_void_p,
+                                 c_void_p, POINTER(moe_plan_t), c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_shared_expert": (c_int32, [c_void_p, POINTER(moe_experts_w), POINTER(moe_dims), c_void_p, c_void_p,
+                                    c_size_t, c_void_p]),
     "moe_forward_host": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float,
                                    c_float, c_float, POINTER(moe_experts_w), c_void_p, c_void_p,
                                    POINTER(moe_plan_t), c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),

@@ -17,7 +17,8 @@ from .abi import check, load
 
 __all__ = [
     "ExpertWeights", "Plan", "moe_workspace_bytes", "moe_workspace_layout", "moe_route", "moe_plan",
-    "moe_experts", "moe_forward", "moe_forward_host", "moe_set_dispatch", "moe_set_combine", "moe_device_error",
+    "moe_experts", "moe_forward", "moe_forward_host", "moe_shared_expert", "moe_set_dispatch", "moe_set_combine",
+    "moe_device_error",
     "moe_last_error", "moe_version", "new_plan", "new_workspace", "dims", "moe_profile_hook",
     "moe_last_launch_count",
 ]
@@ -149,7 +150,7 @@ def moe_experts(x, plan: Plan, topk_w, W: ExpertWeights, *, E: int, I: int, out_
 def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int, k: int, I: int,
                 logits=None, eps: float = 1e-6, router_scale: float = 1.0, out_scale: float = 1.0,
                 topk_idx=None, topk_w=None, plan: Optional[Plan] = None, y=None, ws=None, stream=None,
-                score: str = "sigmoid", norm_topk: bool = True):
+                score: str = "sigmoid", norm_topk: bool = True, y_shared=None):
     T, H = x.shape
     d = abi.moe_dims(T, H, E, k, I)
     dev = x.device
@@ -160,10 +161,22 @@ def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int,
     ws = ws if ws is not None else new_workspace(d, W.fmt, dev)
     cp, cw, rc = plan.c_struct(), W.c_struct(), router_cfg(score, norm_topk)
     check(load().moe_forward_ex(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d), eps,
-                                router_scale, out_scale, ctypes.byref(rc), ctypes.byref(cw), _ptr(topk_idx),
-                                _ptr(topk_w), ctypes.byref(cp), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)),
-          "moe_forward")
+                                router_scale, out_scale, ctypes.byref(rc), _ptr(y_shared), ctypes.byref(cw),
+                                _ptr(topk_idx), _ptr(topk_w), ctypes.byref(cp), _ptr(y), _ptr(ws), ws.numel(),
+                                _stream(stream)), "moe_forward")
     return y, topk_idx, topk_w, plan
+
+
+def moe_shared_expert(x, Ws: ExpertWeights, *, I: int, y_shared=None, ws=None, stream=None):
+    """fp32 (T, H) output of the shared expert (one expert, weight 1, on every token)."""
+    T, H = x.shape
+    d = abi.moe_dims(T, H, 1, 1, I)
+    y_shared = y_shared if y_shared is not None else torch.empty((T, H), dtype=torch.float32, device=x.device)
+    ws = ws if ws is not None else new_workspace(d, Ws.fmt, x.device)
+    cw = Ws.c_struct()
+    check(load().moe_shared_expert(_ptr(x), ctypes.byref(cw), ctypes.byref(d), _ptr(y_shared), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "moe_shared_expert")
+    return y_shared
 
 
 def moe_forward_host(x_host: torch.Tensor, x_dev, W: ExpertWeights, w_router, expert_bias, *, E: int, k: int,

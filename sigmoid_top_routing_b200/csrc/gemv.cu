@@ -14,6 +14,8 @@
 //
 // Work is spread as units of (active expert, 8 rows) over a persistent grid;
 // each CTA takes a contiguous range of units, so most CTAs see one expert.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "launch.h"
@@ -189,12 +191,20 @@ __global__ void __launch_bounds__(256) k_finalize(ExpertArgs a) {
     uint4* dst = reinterpret_cast<uint4*>(a.y);
     const float sc = a.out_scale;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (size_t)gridDim.x * blockDim.x) {
-        const float4 v0 = src[2 * i], v1 = src[2 * i + 1];
+        float4 v0 = src[2 * i], v1 = src[2 * i + 1];
+        v0 = make_float4(__fmul_rn(sc, v0.x), __fmul_rn(sc, v0.y), __fmul_rn(sc, v0.z), __fmul_rn(sc, v0.w));
+        v1 = make_float4(__fmul_rn(sc, v1.x), __fmul_rn(sc, v1.y), __fmul_rn(sc, v1.z), __fmul_rn(sc, v1.w));
+        if (a.y_shared) {   // the shared expert's output, after the routed scale (vllm.cpp PR #684)
+            const float4 s0 = reinterpret_cast<const float4*>(a.y_shared)[2 * i];
+            const float4 s1 = reinterpret_cast<const float4*>(a.y_shared)[2 * i + 1];
+            v0 = make_float4(v0.x + s0.x, v0.y + s0.y, v0.z + s0.z, v0.w + s0.w);
+            v1 = make_float4(v1.x + s1.x, v1.y + s1.y, v1.z + s1.z, v1.w + s1.w);
+        }
         uint4 o;
-        o.x = pack_bf16x2(sc * v0.x, sc * v0.y);
-        o.y = pack_bf16x2(sc * v0.z, sc * v0.w);
-        o.z = pack_bf16x2(sc * v1.x, sc * v1.y);
-        o.w = pack_bf16x2(sc * v1.z, sc * v1.w);
+        o.x = pack_bf16x2(v0.x, v0.y);
+        o.y = pack_bf16x2(v0.z, v0.w);
+        o.z = pack_bf16x2(v1.x, v1.y);
+        o.w = pack_bf16x2(v1.z, v1.w);
         dst[i] = o;
     }
     pdl_trigger();
@@ -218,10 +228,33 @@ __global__ void __launch_bounds__(256) k_finalize_ordered(ExpertArgs a) {
             s.z += v.z;
             s.w += v.w;
         }
+        s = make_float4(__fmul_rn(sc, s.x), __fmul_rn(sc, s.y), __fmul_rn(sc, s.z), __fmul_rn(sc, s.w));
+        if (a.y_shared) {
+            const float4 sh = reinterpret_cast<const float4*>(a.y_shared)[i];
+            s = make_float4(s.x + sh.x, s.y + sh.y, s.z + sh.z, s.w + sh.w);
+        }
         uint2 o;
-        o.x = pack_bf16x2(sc * s.x, sc * s.y);
-        o.y = pack_bf16x2(sc * s.z, sc * s.w);
+        o.x = pack_bf16x2(s.x, s.y);
+        o.y = pack_bf16x2(s.z, s.w);
         reinterpret_cast<uint2*>(a.y)[i] = o;
+    }
+    pdl_trigger();
+}
+
+__global__ void __launch_bounds__(256) k_shared_prep(int T, float* ones, int32_t* counts, int32_t* offsets,
+                                                     int32_t* perm, int32_t* inv, int32_t* tiles) {
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < T; i += gridDim.x * blockDim.x) {
+        ones[i] = 1.0f;
+        perm[i] = i;
+        inv[i] = i;
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        counts[0] = T;
+        offsets[0] = 0;
+        offsets[1] = T;
+        tiles[0] = 0;
+        tiles[1] = (T + kTileM - 1) / kTileM;
     }
     pdl_trigger();
 }
@@ -263,6 +296,12 @@ cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     size_t blocks = (n8 + 255) / 256;
     size_t cap = (size_t)di.sm_count * 8;
     return launch_k(k_finalize, dim3((unsigned)(blocks < cap ? blocks : cap)), dim3(256), 0, s, pdl, a);
+}
+
+cudaError_t launch_shared_prep(int T, float* ones, int32_t* counts, int32_t* offsets, int32_t* perm,
+                               int32_t* inv, int32_t* tiles, bool pdl, cudaStream_t s) {
+    const int blocks = std::max(1, std::min((T + 255) / 256, device_info().sm_count * 4));
+    return launch_k(k_shared_prep, dim3(blocks), dim3(256), 0, s, pdl, T, ones, counts, offsets, perm, inv, tiles);
 }
 
 cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s) {

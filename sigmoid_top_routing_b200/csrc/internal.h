@@ -60,6 +60,7 @@ struct ExpertArgs {
     float* y_acc;            // (T, H) fp32, or (P, H) weighted slot outputs when ordered
     int ordered;             // 1: down stores w * o per plan slot; finalize sums slots in order
     uint16_t* y;             // (T, H) bf16
+    const float* y_shared;   // (T, H) fp32 shared-expert output added after the routed scale, or null
     float out_scale;
     int* err;
 };
@@ -94,6 +95,11 @@ cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // order, filled by launch_gather_x before it.
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// The one-expert identity plan of the shared expert: counts = {T},
+// offsets = {0, T}, perm = inv = 0..T-1, tiles = {0, ceil(T / 128)}, and
+// routing weights of 1.
+cudaError_t launch_shared_prep(int T, float* ones, int32_t* counts, int32_t* offsets, int32_t* perm,
+                               int32_t* inv, int32_t* tiles, bool pdl, cudaStream_t s);
 cudaError_t launch_zero(float* p, size_t n, bool pdl, cudaStream_t s);
 
 // Largest T for which the route kernels run the fused single-CTA select+plan.

@@ -415,17 +415,18 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
                        float out_scale, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
                        const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
-    return moe_forward_ex(x, logits, w_router, expert_bias, d, eps, router_scale, out_scale, nullptr, W,
-                          topk_idx, topk_w, plan, y, ws, ws_bytes, stream);
+    return moe_forward_ex(x, logits, w_router, expert_bias, d, eps, router_scale, out_scale, nullptr, nullptr,
+                          W, topk_idx, topk_w, plan, y, ws, ws_bytes, stream);
 }
 
 moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
                           const float* expert_bias, const moe_dims* d, float eps, float router_scale,
-                          float out_scale, const moe_router_cfg* cfg, const moe_experts_w* W,
-                          int32_t* topk_idx, float* topk_w, const moe_plan_t* plan, void* y, void* ws,
-                          size_t ws_bytes, moe_stream_t stream) {
+                          float out_scale, const moe_router_cfg* cfg, const float* y_shared,
+                          const moe_experts_w* W, int32_t* topk_idx, float* topk_w, const moe_plan_t* plan,
+                          void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    if (y_shared && !aligned16(y_shared)) return fail(MOE_ERR_ALIGN, "y_shared not 16-byte aligned");
     RouteArgs r0{};
     if ((st = check_router_cfg(cfg, &r0)) != MOE_OK) return st;
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
@@ -473,8 +474,51 @@ moe_status moe_forward_ex(const void* x, const float* logits, const float* w_rou
         e = q.stage(MOE_STAGE_PLAN, [&](int* n) { return launch_plan(p, true, q.s, n); });
         if (e != cudaSuccess) return cuda_fail(e, "plan");
     }
-    const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    a.y_shared = y_shared;
     if ((st = run_experts(q, a, d)) != MOE_OK) return st;
+    g_launches = q.n;
+    return MOE_OK;
+}
+
+moe_status moe_shared_expert(const void* x, const moe_experts_w* Ws, const moe_dims* d, float* y_shared,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status st = check_dims(d);
+    if (st != MOE_OK) return st;
+    if (d->E != 1 || d->k != 1) return fail(MOE_ERR_SHAPE, "the shared expert needs E == 1 and k == 1");
+    if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
+    if (!x || !y_shared) return fail(MOE_ERR_NULL, "x or y_shared is NULL");
+    if (!aligned16(x) || !aligned16(y_shared)) return fail(MOE_ERR_ALIGN, "x or y_shared not 16-byte aligned");
+    if ((st = check_weights(Ws)) != MOE_OK) return st;
+    WsView v;
+    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    // the identity plan and the weights of 1 live in the scratch region (at
+    // E = 1 it holds >= 4224 + 32 T bytes, more than the 3 align256(4 T) + 48
+    // used here); x is already in plan order, so nothing is gathered
+    const size_t T = d->T;
+    char* b = reinterpret_cast<char*>(v.l_scratch);
+    float* ones = reinterpret_cast<float*>(b);
+    int32_t* perm = reinterpret_cast<int32_t*>(b + align256(T * 4));
+    int32_t* inv = reinterpret_cast<int32_t*>(b + 2 * align256(T * 4));
+    int32_t* misc = reinterpret_cast<int32_t*>(b + 3 * align256(T * 4));   // counts[1] | offsets[2] | tiles[2]
+    moe_plan_t plan{misc, misc + 4, perm, inv, misc + 8};
+    Seq q{reinterpret_cast<cudaStream_t>(stream)};
+    cudaError_t e = launch_shared_prep(d->T, ones, plan.counts, plan.offsets, perm, inv, plan.tiles, true, q.s);
+    if (e != cudaSuccess) return cuda_fail(e, "shared-expert plan");
+    q.n = 1;
+    ExpertArgs a = make_expert_args(x, &plan, ones, d, Ws, 1.0f, nullptr, v);
+    a.xs = static_cast<uint16_t*>(const_cast<void*>(x));
+    a.y_acc = y_shared;
+    if (!a.ordered) {
+        if ((e = launch_zero(y_shared, T * d->H, true, q.s)) != cudaSuccess) return cuda_fail(e, "zero y_shared");
+        ++q.n;
+    }
+    const bool gemv = use_gemv(d, a.fmt);
+    e = q.stage(MOE_STAGE_UP, [&](int*) { return gemv ? launch_gemv_up(a, true, q.s) : launch_gemm_up(a, true, q.s); });
+    if (e == cudaErrorNotSupported) return fail(MOE_ERR_UNSUPPORTED, "no expert kernel for this format/path");
+    if (e != cudaSuccess) return cuda_fail(e, "shared expert up kernel");
+    e = q.stage(MOE_STAGE_DOWN, [&](int*) { return gemv ? launch_gemv_down(a, true, q.s) : launch_gemm_down(a, true, q.s); });
+    if (e != cudaSuccess) return cuda_fail(e, "shared expert down kernel");
     g_launches = q.n;
     return MOE_OK;
 }

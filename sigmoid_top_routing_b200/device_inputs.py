@@ -47,6 +47,22 @@ def to_device(inp: MoEInputs, device="cuda", with_x: bool = True) -> DeviceInput
                         expert_bias=torch.from_numpy(inp.expert_bias).to(device), W=W)
 
 
+def shared_to_device(inp: MoEInputs, device="cuda") -> Optional[ExpertWeights]:
+    """The shared expert's weights (None when the workload has none)."""
+    wl, sh = inp.wl, inp.shared
+    if not sh:
+        return None
+    act = abi.MOE_ACT_SWIGLU if wl.act == "swiglu" else abi.MOE_ACT_RELU2
+    if wl.fmt == "bf16":
+        return ExpertWeights(act=act, fmt=abi.MOE_W_BF16, w1=bf16_tensor(sh["w1_bits"], device),
+                             w2=bf16_tensor(sh["w2_bits"], device), swiglu_limit=wl.swiglu_limit)
+    return ExpertWeights(act=act, fmt=abi.MOE_W_AFFINE4_G64,
+                         w1=u32_tensor(sh["w1_q"], device), w2=u32_tensor(sh["w2_q"], device),
+                         w1_scale=bf16_tensor(sh["w1_scale"], device), w1_bias=bf16_tensor(sh["w1_bias"], device),
+                         w2_scale=bf16_tensor(sh["w2_scale"], device), w2_bias=bf16_tensor(sh["w2_bias"], device),
+                         swiglu_limit=wl.swiglu_limit)
+
+
 def weight_bytes(inp: MoEInputs, experts) -> int:
     """Bytes of the given experts' weights (codes, scales and biases included)."""
     wl = inp.wl

@@ -155,8 +155,20 @@ def test_router_cfg_refuses_unknown_modes(lib):
         assert lib.moe_route_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, ctypes.byref(cfg),
                                 0x30000, 0x40000, None) == abi.MOE_ERR_UNSUPPORTED
         assert lib.moe_forward_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, 1.0,
-                                  ctypes.byref(cfg), ctypes.byref(_weights()), 0x30000, 0x40000,
+                                  ctypes.byref(cfg), None, ctypes.byref(_weights()), 0x30000, 0x40000,
                                   ctypes.byref(_plan()), 0x50000, 0x1000000, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+
+
+def test_shared_expert_refuses_bad_shapes(lib):
+    W = _weights()
+    for d in (_d(E=2, k=1), _d(E=4, k=2)):
+        assert lib.moe_shared_expert(0x10000, ctypes.byref(W), ctypes.byref(d), 0x20000, 0x1000000, 1 << 30,
+                                     None) == abi.MOE_ERR_SHAPE
+    d = _d(E=1, k=1)
+    assert lib.moe_shared_expert(0x10000, ctypes.byref(W), ctypes.byref(d), None, 0x1000000, 1 << 30,
+                                 None) == abi.MOE_ERR_NULL
+    assert lib.moe_shared_expert(0x10000, ctypes.byref(W), ctypes.byref(d), 0x20004, 0x1000000, 1 << 30,
+                                 None) == abi.MOE_ERR_ALIGN
 
 
 def test_forward_refuses_missing_router(lib):

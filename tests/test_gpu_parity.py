@@ -49,9 +49,13 @@ def run_forward(api, inp, *, dispatch=None, logits=None, poison=True):
                       plan.tiles):
                 t.view(torch.uint8).fill_(0xFF)
         lg = None if logits is None else torch.from_numpy(logits).cuda()
+        y_sh = None
+        if wl.shared_I:
+            from sigmoid_top_routing_b200.device_inputs import shared_to_device
+            y_sh = api.moe_shared_expert(D.x, shared_to_device(inp), I=wl.shared_I)
         api.moe_forward(D.x, D.W, D.w_router, D.expert_bias, E=wl.E, k=wl.k, I=wl.I, logits=lg,
                         eps=wl.eps, router_scale=wl.router_scale, out_scale=wl.out_scale, topk_idx=idx,
-                        topk_w=w, plan=plan, y=y, ws=ws, score=wl.score, norm_topk=wl.norm_topk)
+                        topk_w=w, plan=plan, y=y, ws=ws, score=wl.score, norm_topk=wl.norm_topk, y_shared=y_sh)
         torch.cuda.synchronize()
         assert api.moe_device_error() == 0
     finally:
