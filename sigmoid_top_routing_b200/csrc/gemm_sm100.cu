@@ -553,14 +553,18 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 if (MODE == kDown) {
                     const int f = tl.wt * 128 + lrow;
                     if (!dead && f < g.feats) {
+                        if (!g.ordered) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int c = c0 + i;
-                            if (c >= tl.ntok) continue;
-                            if (g.ordered)
-                                __stcg(g.y_acc + (size_t)(tl.row0 + c) * g.H + f, s_tokw[c] * v[i]);
-                            else
-                                red_add_f32(g.y_acc + (size_t)s_tok[c] * g.H + f, s_tokw[c] * v[i]);
+                            for (int i = 0; i < 16; ++i) {
+                                const int c = c0 + i;
+                                if (c < tl.ntok) red_add_f32(g.y_acc + (size_t)s_tok[c] * g.H + f, s_tokw[c] * v[i]);
+                            }
+                        } else {   // one store per slot row (plan order)
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const int c = c0 + i;
+                                if (c < tl.ntok) __stcg(g.y_acc + (size_t)(tl.row0 + c) * g.H + f, s_tokw[c] * v[i]);
+                            }
                         }
                     }
                 } else if (MODE == kUpRelu2) {
