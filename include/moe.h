@@ -264,10 +264,8 @@ MOE_API int32_t moe_last_launch_count(void);
 /* moe_forward for callers that cannot allocate device memory.  (The pages
  * have no counterpart: this is an interface choice of this library.)
  * Some callers have no workspace to give: a plugin host that hands a custom
- * op only its input and output tensors, code running inside another
- * framework's CUDA-graph capture (where cudaMalloc cannot be captured and may
- * synchronise the device), or a latency-bound serving loop that must never
- * wait on an allocator.  This call takes the same arguments as moe_forward
+ * op only its input and output tensors, or a latency-bound serving loop that
+ * must never wait on an allocator.  This call takes the same arguments as moe_forward
  * minus ws/ws_bytes: its scratch (fp32 accumulator, bf16 activations, router
  * logits) is one fixed 16 MiB device array inside the library, which every GPU
  * that loads the library holds until the process exits.  It allocates
@@ -277,8 +275,7 @@ MOE_API int32_t moe_last_launch_count(void);
  *     message giving the bytes needed.  Runs bf16 weights only, always on the
  *     weight-streaming grouped GEMV (MOE_ERR_UNSUPPORTED for affine 4-bit).
  *   - The first call on a device looks up the array's device address on that
- *     device (cudaGetSymbolAddress, once per device, with the device current);
- *     make that first call before any stream capture.
+ *     device (cudaGetSymbolAddress, once per device, with the device current).
  *   - Every call shares the array and it keeps the last call's contents (the
  *     accumulator is cleared at the start of each call).  Calls whose work
  *     overlaps on the GPU (other streams, other threads) race on it: run them

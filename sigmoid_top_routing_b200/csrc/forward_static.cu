@@ -2,13 +2,11 @@
 // allocate device memory.
 //
 // Some callers have no way to hand the library a workspace: a plugin host
-// that gives a custom op only its input and output tensors, code that runs
-// inside another framework's CUDA-graph capture (where cudaMalloc is not a
-// capturable operation and may synchronise the device), or a latency-bound
-// serving loop that must never wait on an allocator.  For them the scratch
-// the forward needs (the fp32 accumulator, the bf16 activations and the
-// router-logit scratch) lives in one fixed device array defined in this
-// file.  The caller still passes the inputs, the weights, the plan arrays
+// that gives a custom op only its input and output tensors, or a
+// latency-bound serving loop that must never wait on an allocator.  For them
+// the scratch the forward needs (the fp32 accumulator, the bf16 activations
+// and the router-logit scratch) lives in one fixed device array defined in
+// this file.  The caller still passes the inputs, the weights, the plan arrays
 // and the outputs; this entry point calls no cudaMalloc, cudaFree or any
 // allocating library routine.
 #include <cstdio>

@@ -1,7 +1,6 @@
 """moe_forward_static, the forward pass for callers that cannot allocate
 device memory (a plugin host that only hands over input and output tensors,
-code inside another framework's graph capture, a serving loop that must not
-wait on an allocator).  It keeps its scratch in a fixed array inside the
+a serving loop that must not wait on an allocator).  It keeps its scratch in a fixed array inside the
 library instead of a caller workspace.
 
 Called here through the C ABI, twice in a row (the array keeps the previous
