@@ -14,8 +14,9 @@
 // (Sx from an all-ones A operand on the same x fragments).  The group's scale
 // and bias are then applied in fp32:
 //     sum_k w[r][k] x[n][k] = s * Sq + (b - 128 s) * Sx.
-// The MMA is only a dot-product engine here (N = 8 token columns); the kernel
-// is bound by the code stream, not by tensor throughput.
+// The MMA is only a dot-product engine here (N = 8 token columns); tensor
+// throughput does not bound the kernel (as measured it is issue-bound, about
+// four instructions per weight).
 //
 // Within one MMA the k order is free as long as A and B agree: a lane's word
 // of 8 nibbles covers k0..k0+7, and the A slots (2t, 2t+1) / (2t+8, 2t+9) of
@@ -29,10 +30,13 @@
 //
 //   up   (SwiGLU): h[slot, i] = bf16_rn(silu(g) * u)
 //   up   (relu^2): h[slot, i] = bf16_rn(relu(u)^2)
-//   down:          y_acc[t, n] += w[pair] * (W2[e][n] . h[slot])   (fp32 atomics)
+//   down:          y_acc[t, n] += w[pair] * (W2[e][n] . h[slot])   (fp32 atomics;
+//                  a plain store per plan slot under the ordered combine)
 //
-// Units are (active expert, 16-row block, chunk of <= 8 of its tokens), one
-// per warp; warps never wait on one another.
+// A CTA of 4 warps takes a unit (active expert, chunk of <= 8 of its tokens,
+// 4 consecutive 16-row blocks -- one per warp): the chunk's token rows are
+// copied into shared memory once by cp.async while the warps' code rings are
+// already in flight, and the warps meet at one barrier per unit.
 #include "common.cuh"
 #include "internal.h"
 #include "launch.h"
