@@ -512,9 +512,19 @@ def main():
     return 0
 
 
+def code_hash(text: str) -> str:
+    """sha256 prefix of C++ source with comments and whitespace removed: a
+    comment edit leaves it unchanged, any code change moves it."""
+    import hashlib
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()[:16]
+
+
 def traffic_of(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of that kernel; else None."""
+    the current code of that kernel's source file; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -524,10 +534,9 @@ def traffic_of(kernel: str, workload: str):
         rec = d.get(f"{kernel}:{workload}")
         if not rec:
             return None
-        import hashlib
         src = os.path.join(ROOT, "sigmoid_top_routing_b200", "csrc", rec["source"])
-        with open(src, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+        with open(src) as f:
+            if code_hash(f.read()) != rec["code_sha256_16"]:
                 return None
         return rec["bytes_per_launch"]
     except Exception:

@@ -7,14 +7,19 @@
 // tiles.  D[feature][token] accumulates in fp32 in TMEM (double-buffered so
 // the epilogue overlaps the next tile's main loop).
 //
-//   up (SwiGLU):  a tile = 64 gate rows + 64 up rows of W1[e] (gate-first
-//                 layout, TileGym PR #187 "Weight layout and routing"); TMEM
-//                 lanes j and 64 + j hold gate and up of feature j, and the
-//                 epilogue writes h[pos, f] = bf16_rn(silu(g) * u).
+//   up (SwiGLU):  gate-first W1[e] (TileGym PR #187 "Weight layout and
+//                 routing").  Token tiles of 32: a tile = 64 gate rows + the
+//                 64 matching up rows, TMEM lanes j and 64 + j hold gate and up
+//                 of feature j and the halves meet through shared memory;
+//                 tiles of 64 or more: 128 gate + 128 up rows in two TMEM
+//                 accumulators.  The epilogue clamps the inputs when
+//                 swiglu_limit > 0 and writes h[pos, f] = bf16_rn(silu(g) * u).
 //   up (relu^2):  a tile = 128 rows of W1[e]; h = bf16_rn(relu(u)^2), NaN
 //                 kept (vllm.cpp PR #684; bloomery PR #235 "What").
 //   down:         a tile = 128 rows of W2[e]; y_acc[t, f] += w[p] * D (fp32
-//                 reductions), the weighted combine of the pages' MoeCombine.
+//                 reductions), the weighted combine of the pages' MoeCombine;
+//                 under the ordered combine, one store of w[p] * D per plan
+//                 slot instead.
 //
 // Prior art: the staged prompt kernels of TensorFold issue #548 ("Prompt rows
 // of the grouped experts: two forms": items of 64 pairs x 128 columns staged

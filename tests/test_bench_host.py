@@ -78,3 +78,11 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
     args = b.parse()
     assert b.run_reference(args) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_code_hash_ignores_comments_but_not_code():
+    b = _bench()
+    src = "int f(int a) {\n    return a + 1;   // one more\n}\n/* block\n comment */\n"
+    assert b.code_hash(src) == b.code_hash("int f(int a) { return a + 1; }")
+    assert b.code_hash(src) == b.code_hash(src.replace("one more", "the next integer"))
+    assert b.code_hash(src) != b.code_hash(src.replace("a + 1", "a + 2"))
