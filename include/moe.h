@@ -22,6 +22,12 @@
  *            multiplies the finished sum once (vllm.cpp PR #684, "The finding
  *            that justifies the row").
  *
+ * Variants, each declared below with its passage: softmax router scores and
+ * norm_topk off (moe_router_cfg, moe_route_ex / moe_forward_ex), the SwiGLU
+ * input clamp (moe_experts_w.swiglu_limit), a shared expert added after the
+ * routed scale (moe_shared_expert, moe_forward_ex's y_shared), and a
+ * slot-ordered, batch-invariant combine (moe_set_combine).
+ *
  * Conventions for every entry point
  *   - Pointers named x, logits, w_router, expert_bias, topk_*, plan arrays,
  *     weights, y and ws are DEVICE pointers (the caller owns the memory; the
