@@ -86,3 +86,27 @@ def test_code_hash_ignores_comments_but_not_code():
     assert b.code_hash(src) == b.code_hash("int f(int a) { return a + 1; }")
     assert b.code_hash(src) == b.code_hash(src.replace("one more", "the next integer"))
     assert b.code_hash(src) != b.code_hash(src.replace("a + 1", "a + 2"))
+
+
+def test_work_model_counts_each_tensor_once():
+    """Algorithmic bytes / FLOPs of the decode workload, written out by hand:
+    the up kernel streams each active expert's gate_up once (2I x H bf16)
+    plus x and h; the step adds the down weights, the router, h twice, the
+    fp32 accumulator three times and y."""
+    b = _bench()
+    from sigmoid_top_routing_b200 import inputs as G
+    wl = G.WORKLOADS["lfm2_decode_t8"]
+    inp = G.make_inputs(wl, with_experts=False)
+    counts = [0] * wl.E
+    for e in (0, 3, 5):
+        counts[e] = 2
+    m = b.work_model(inp, counts)
+    T, H, E, k, I = wl.T, wl.H, wl.E, wl.k, wl.I
+    P = T * k
+    assert m["active_experts"] == 3
+    assert m["w1_bytes_per_expert"] == 2 * I * H * 2
+    assert m["up_bytes"] == 3 * 2 * I * H * 2 + T * H * 2 + P * I * 2
+    assert m["up_flops"] == 2.0 * P * 2 * I * H
+    assert m["flops"] == 2.0 * P * (2 * I * H + H * I)
+    assert m["step_bytes"] == (3 * (2 * I * H + H * I) * 2 + T * H * 2 + E * H * 4 + 2 * P * I * 2
+                               + 3 * T * H * 4 + T * H * 2)
