@@ -91,11 +91,12 @@ moe_status check_fmt(int32_t fmt) {
     return MOE_OK;
 }
 
-void layout(const moe_dims* d, moe_ws_layout* L) {
+// ordered: the combine mode the call runs with (read once per call)
+void layout(const moe_dims* d, moe_ws_layout* L, bool ordered) {
     const size_t T = d->T, H = d->H, E = d->E, P = (size_t)d->T * d->k, I = d->I;
     size_t off = 0;
     L->y_acc = off;       // (T, H) sums, or (P, H) slot outputs for the ordered combine
-    off = align256(off + (combine_ordered() ? P : T) * H * 4);
+    off = align256(off + (ordered ? P : T) * H * 4);
     L->h = off;
     off = align256(off + P * I * 2);
     L->xs = off;          // token rows gathered in plan order (wide token tiles)
@@ -114,11 +115,13 @@ struct WsView {
     float* l_scratch;
     int32_t* plan_scratch;
     float* part;
+    bool ordered;            // the combine mode of this call (read once)
 };
 
 moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
     moe_ws_layout L;
-    layout(d, &L);
+    v->ordered = combine_ordered();
+    layout(d, &L, v->ordered);
     if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_ALIGN, "workspace not 256-byte aligned");
     if (ws_bytes < L.total)
@@ -229,7 +232,7 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.h = v.h;
     a.xs = v.xs;
     a.y_acc = v.y_acc;
-    a.ordered = combine_ordered() ? 1 : 0;
+    a.ordered = v.ordered ? 1 : 0;
     a.y = static_cast<uint16_t*>(y);
     a.out_scale = out_scale;
     a.err = device_info().err_word;
@@ -321,7 +324,7 @@ extern "C" {
 size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt) {
     if (check_dims(d) != MOE_OK || check_fmt(fmt) != MOE_OK) return 0;
     moe_ws_layout L;
-    layout(d, &L);
+    layout(d, &L, combine_ordered());
     return L.total;
 }
 
@@ -330,7 +333,7 @@ moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* o
     if (st != MOE_OK) return st;
     if ((st = check_fmt(fmt)) != MOE_OK) return st;
     if (!out) return fail(MOE_ERR_NULL, "out is NULL");
-    layout(d, out);
+    layout(d, out, combine_ordered());
     return MOE_OK;
 }
 
@@ -462,7 +465,7 @@ moe_status moe_forward_ex(const void* x, const float* logits, const float* w_rou
     r.perm = plan->perm;
     r.inv = plan->inv;
     r.tiles = plan->tiles;
-    r.zero_ptr = combine_ordered() ? nullptr : v.y_acc;   // the router also clears the accumulator
+    r.zero_ptr = v.ordered ? nullptr : v.y_acc;   // the router also clears the accumulator
     r.zero_count = (size_t)d->T * d->H;
     r.err = device_info().err_word;
     const bool fuse = d->T <= kSmallT;  // one CTA routes and plans all pairs
