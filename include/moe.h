@@ -161,7 +161,7 @@ typedef struct {
     size_t y_acc;   /* fp32 (T, H): the unscaled routed sum; (P, H) weighted slot outputs
                        under MOE_COMBINE_ORDERED */
     size_t h;       /* bf16 (P, I): activations in plan order */
-    size_t xs;      /* bf16 (P, H): token rows gathered in plan order (wide token tiles) */
+    size_t xs;      /* bf16 (P, H): token rows gathered in plan order (tcgen05 GEMM path) */
     size_t scratch; /* plan and scheduler scratch */
     size_t total;   /* == moe_workspace_bytes() */
 } moe_ws_layout;

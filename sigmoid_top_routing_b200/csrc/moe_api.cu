@@ -99,7 +99,7 @@ void layout(const moe_dims* d, moe_ws_layout* L, bool ordered) {
     off = align256(off + (ordered ? P : T) * H * 4);
     L->h = off;
     off = align256(off + P * I * 2);
-    L->xs = off;          // token rows gathered in plan order (wide token tiles)
+    L->xs = off;          // token rows gathered in plan order (the up GEMM reads them by TMA)
     off = align256(off + P * H * 2);
     // scratch: router logits (T <= 32) | plan histograms and bases | per-segment partial logits
     L->scratch = off;
