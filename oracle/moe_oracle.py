@@ -34,7 +34,7 @@ What it computes, and where each step is stated:
              dequantised exactly in float64 as in its "Verification" section
              (the float64 reference dequantises the MLX weights exactly).
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * the bias is added to the sigmoid score, c = s + b, for selection only;
   * selection order: descending c, ties to the lower expert index, NaN below
     every number, -0.0 == +0.0; the k picks are returned in rank order;

@@ -71,10 +71,8 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
                                          float router_scale, float out_scale, const moe_experts_w* W,
                                          int32_t* topk_idx, float* topk_w, const moe_plan_t* plan,
                                          void* y, moe_stream_t stream) {
-    if (!d) return fail(MOE_ERR_NULL, "dims is NULL");
-    if (d->T < 0 || d->H < 64 || d->H > 16384 || d->H % 64 || d->I < 64 || d->I > 16384 || d->I % 64 ||
-        d->E < 1 || d->E > 256 || d->k < 1 || d->k > d->E || d->k > 32)
-        return fail(MOE_ERR_SHAPE, "sizes out of range (see moe_dims)");
+    moe_status st = validate_dims(d);
+    if (st != MOE_OK) return st;
     if (d->T == 0) {
         set_last_launch_count(0);
         return MOE_OK;
@@ -83,15 +81,9 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
     if (!logits && !w_router) return fail(MOE_ERR_NULL, "w_router is NULL (routing from x)");
     if (!aligned16(x) || !aligned16(y) || (!logits && !aligned16(w_router)))
         return fail(MOE_ERR_ALIGN, "x, y or w_router not 16-byte aligned");
-    if (!plan || !plan->counts || !plan->offsets || !plan->perm || !plan->inv || !plan->tiles)
-        return fail(MOE_ERR_NULL, "plan or a plan array is NULL");
-    if (!W || !W->w1 || !W->w2) return fail(MOE_ERR_NULL, "weights are NULL");
+    if ((st = validate_plan(plan)) != MOE_OK) return st;
+    if ((st = validate_weights(W)) != MOE_OK) return st;
     if (W->fmt != MOE_W_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_forward_static runs bf16 weights only");
-    if (W->act != MOE_ACT_SWIGLU && W->act != MOE_ACT_RELU2)
-        return fail(MOE_ERR_UNSUPPORTED, "unknown activation");
-    if (!aligned16(W->w1) || !aligned16(W->w2)) return fail(MOE_ERR_ALIGN, "w1/w2 not 16-byte aligned");
-    if (!(W->swiglu_limit >= 0.0f) || W->swiglu_limit > 3.0e38f)
-        return fail(MOE_ERR_SHAPE, "swiglu_limit must be finite and >= 0 (0 = off)");
 
     // scratch layout: y_acc fp32 (T, H) | h bf16 (P, I) | router-logit scratch
     const size_t T = d->T, H = d->H, I = d->I, E = d->E, P = T * d->k;

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 struct RouteArgs {
@@ -108,5 +110,10 @@ constexpr int kSmallT = 32;
 // Thread-local status text and launch count of the C-ABI layer (moe_api.cu).
 void set_last_error(const char* msg);
 void set_last_launch_count(int n);
+// The C-ABI layer's argument checks, shared by every entry point: on failure
+// they set the thread's status text and return the status.
+moe_status validate_dims(const moe_dims* d);          // sizes within moe_dims' limits
+moe_status validate_plan(const moe_plan_t* plan);     // plan struct and its arrays non-NULL
+moe_status validate_weights(const moe_experts_w* W);  // pointers, alignment, enums, swiglu_limit
 
 }  // namespace moe

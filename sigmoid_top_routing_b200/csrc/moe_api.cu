@@ -317,6 +317,9 @@ namespace moe {
 // For entry points defined in other files of the library.
 void set_last_error(const char* msg) { g_last_error = msg; }
 void set_last_launch_count(int n) { g_launches = n; }
+moe_status validate_dims(const moe_dims* d) { return check_dims(d); }
+moe_status validate_plan(const moe_plan_t* plan) { return check_plan(plan); }
+moe_status validate_weights(const moe_experts_w* W) { return check_weights(W); }
 }  // namespace moe
 
 extern "C" {

@@ -110,3 +110,68 @@ def test_work_model_counts_each_tensor_once():
     assert m["flops"] == 2.0 * P * (2 * I * H + H * I)
     assert m["step_bytes"] == (3 * (2 * I * H + H * I) * 2 + T * H * 2 + E * H * 4 + 2 * P * I * 2
                                + 3 * T * H * 4 + T * H * 2)
+
+
+def _all_active(wl):
+    return [1] * wl.E
+
+
+@pytest.mark.parametrize("name,bound", [
+    ("lfm2_decode_t8", "hbm"), ("lfm2_prefill_t4096", "tensor"), ("nemotron_relu2_t2048", "hbm"),
+    ("affine4_t1", "hbm"), ("affine4_t8", "hbm"), ("affine4_t64", "hbm"), ("affine4_t512", "hbm"),
+    ("affine4_t8192", "tensor")])
+def test_roofline_bound_of_every_configuration(name, bound):
+    """The up kernel's bound follows from its FLOPs per algorithmic byte
+    against the ridge of the measured peaks (sustained GEMM / HBM copy)."""
+    b = _bench()
+    from sigmoid_top_routing_b200 import inputs as G
+    wl = G.WORKLOADS[name]
+    m = b.work_model(G.make_inputs(wl, with_experts=False), _all_active(wl))
+    pk = {"hbm_gbs": 6548.8, "bf16_tflops": 1628.7, "bf16_tflops_sustained": 1380.3}
+    assert b.ridge_flop_per_byte(pk) == pytest.approx(1380.3e3 / 6548.8)
+    r = b.roofline_of(m, 100.0, pk, "measured", None)
+    assert r["bound"] == bound
+    if bound == "hbm":
+        assert r["achieved"] == pytest.approx(m["up_bytes"] / 100e-6 / 1e9)
+        assert r["peak"] == 6548.8 and r["nominal_peak"] == 7700.0
+    else:
+        assert r["achieved"] == pytest.approx(m["up_flops"] / 100e-6 / 1e12)
+        assert r["peak"] == 1380.3 and r["nominal_peak"] == 2250.0
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+
+
+def test_graph_block_fits_any_step_count():
+    b = _bench()
+    assert b.block_steps(20, 2) == 20
+    assert b.block_steps(100, 2) == 32
+    assert b.block_steps(7, 2) == 6
+    assert b.block_steps(1, 2) == 2          # K < n_sets: only single-step graphs replay
+    assert b.block_steps(40, 3) == 30
+    # the event pairs the last replays of K steps leave behind
+    assert b.replayed_events(20, 20, 20, 2) == [("block", range(20))]
+    assert b.replayed_events(1, 2, 2, 2) == [("single", range(1))]
+    assert b.replayed_events(45, 32, 32, 2) == [("block", range(32)), ("single", range(2))]
+
+
+def test_side_workloads_selection():
+    b = _bench()
+    assert b.side_workloads("none", "lfm2_prefill_t4096") == []
+    allw = b.side_workloads("all", "lfm2_prefill_t4096")
+    assert "lfm2_decode_t8" in allw and "affine4_t8192" in allw and "lfm2_prefill_t4096" not in allw
+    assert b.side_workloads("affine4_t1,lfm2_prefill_t4096", "lfm2_prefill_t4096") == ["affine4_t1"]
+
+
+def test_reference_arm_config_matches_ours(capsys, monkeypatch):
+    """Both arms describe the workload with the same config dict."""
+    import json
+    b = _bench()
+    monkeypatch.delenv("RANK", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "tiny", "--steps", "1",
+                                      "--warmup", "0"])
+    args = b.parse()
+    assert b.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    from sigmoid_top_routing_b200 import inputs as G
+    assert line["config"] == b.config_of(G.WORKLOADS["tiny"], b.parse(["--workload", "tiny"]))
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
