@@ -53,6 +53,15 @@ gate and up pre-activations clamp and limit 0 is the control):
   * swiglu_limit L > 0: g <- min(g, L), u <- clamp(u, -L, L) before
     silu(g) * u, NaN kept (0 turns the clamp off).
 
+Skip slot (TensorFold issue #548, "Paths your experts test does not reach",
+the "skip a slot" row: the block's 9-slot plan is top-8 plus the shared
+expert's id 288, over 289 plan experts, with expert 288 skipped; the result
+equals the 8-slot form and the skipped slot's rows are left untouched):
+  * the plan is built over the plan experts as usual (the skip id is an
+    ordinary expert there);
+  * the expert stage computes nothing for pairs routed to the skip id, and
+    the combine leaves them out: acc = sum over the kept slots, in slot order.
+
 Shared expert (vllm.cpp PR #684, "The finding that justifies the row": the
 combine multiplies the routed sum by the routed scale BEFORE the shared
 expert's output is added; the shared output itself is not scaled):
@@ -67,7 +76,8 @@ __all__ = [
     "bf16_to_f64", "router_logits", "sigmoid", "select_topk", "select_topk_bruteforce",
     "route", "tie_margins", "plan", "dequant_affine4", "silu", "swiglu", "relu2", "softmax",
     "clamp_swiglu_inputs",
-    "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "shared_expert", "BM",
+    "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "shared_expert", "experts_block",
+    "BM",
 ]
 
 BM = 128  # rows of one GEMM M-tile; the plan's tile table counts ceil(count / BM) per expert
@@ -273,16 +283,20 @@ def _act(h1: np.ndarray, act: str, I: int, limit: float = 0.0) -> np.ndarray:
     raise ValueError(act)
 
 
-def expert_outputs(inp, idx: np.ndarray, tokens: np.ndarray) -> np.ndarray:
+def expert_outputs(inp, idx: np.ndarray, tokens: np.ndarray, skip=None) -> np.ndarray:
     """o[r, j, :] = down_e(act(up_e(x_t))) for t = tokens[r], e = idx[r, j].
 
     For each expert, the rows routed to it are stacked and multiplied by its
-    weights (a matmul per expert); nothing else is reordered."""
+    weights (a matmul per expert); nothing else is reordered.  Pairs routed to
+    the expert id ``skip`` are not computed (their o stays 0; the skipped
+    expert has no weights)."""
     wl = inp.wl
     x = bf16_to_f64(inp.x_bits[tokens])
     R, k = idx.shape
     o = np.zeros((R, k, wl.H))
     for e in np.unique(idx):
+        if skip is not None and e == skip:
+            continue
         rr, jj = np.nonzero(idx == e)
         W1 = _expert_w(inp, "w1", int(e))
         W2 = _expert_w(inp, "w2", int(e))
@@ -310,15 +324,19 @@ def shared_expert(inp, tokens: np.ndarray) -> np.ndarray:
         return a @ _shared_w(inp, "w2").T
 
 
-def combine(o: np.ndarray, w: np.ndarray, out_scale: float, dtype=np.float64):
+def combine(o: np.ndarray, w: np.ndarray, out_scale: float, dtype=np.float64, keep=None):
     """acc = sum_j w_j * o_j in slot order, then y = out_scale * acc: one
     multiply on the finished sum (vllm.cpp PR #684).  ``dtype`` float32 gives
-    the fp32 mirror used to pin the order of operations."""
+    the fp32 mirror used to pin the order of operations.  ``keep`` (R, k)
+    bool leaves the unkept slots out of the sum (skip slots)."""
     o = np.asarray(o).astype(dtype)
     w = np.asarray(w).astype(dtype)
     acc = np.zeros(o.shape[0:1] + o.shape[2:], dtype=dtype)
     for j in range(o.shape[1]):
-        acc = acc + w[:, j, None] * o[:, j]
+        term = w[:, j, None] * o[:, j]
+        if keep is not None:
+            term = np.where(np.asarray(keep)[:, j, None], term, dtype(0))
+        acc = acc + term
     return acc, dtype(out_scale) * acc
 
 
@@ -354,6 +372,19 @@ def moe_block(inp, tokens=None, *, use_logits=None, idx=None):
         r["shared"] = sh
     r.update({"tokens": tokens, "acc": acc, "y": y})
     return r
+
+
+def experts_block(inp, idx, w, tokens=None, skip=None):
+    """The expert stage and combine on given picks and weights: for token rows
+    ``tokens`` (default all), idx (R, k) plan-expert ids and w (R, k) weights,
+    returns (acc, y) with the pairs routed to ``skip`` computed nowhere and left
+    out of the sum (the 9-slot plan of TensorFold issue #548: top-8 plus the
+    shared id, that id skipped)."""
+    tokens = np.arange(inp.wl.T) if tokens is None else np.asarray(tokens)
+    idx = np.asarray(idx, dtype=np.int64)
+    o = expert_outputs(inp, idx, tokens, skip=skip)
+    keep = None if skip is None else idx != skip
+    return combine(o, w, inp.wl.out_scale, keep=keep)
 
 
 def moe_block_all_experts(inp):
