@@ -25,8 +25,10 @@
  * Variants, each declared below with its passage: softmax router scores and
  * norm_topk off (moe_router_cfg, moe_route_ex / moe_forward_ex), the SwiGLU
  * input clamp (moe_experts_w.swiglu_limit), a shared expert added after the
- * routed scale (moe_shared_expert, moe_forward_ex's y_shared), and a
- * slot-ordered, batch-invariant combine (moe_set_combine).
+ * routed scale (moe_shared_expert, moe_forward_ex's y_shared), a skipped
+ * plan expert (moe_experts_ex's skip_expert: the 9-slot plan with the shared
+ * expert's id), and a slot-ordered, batch-invariant combine (moe_exec_cfg /
+ * moe_set_combine).
  *
  * Conventions for every entry point
  *   - Pointers named x, logits, w_router, expert_bias, topk_*, plan arrays,
@@ -78,7 +80,8 @@ typedef enum {
 typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act;
 typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1 } moe_wfmt;
 
-/* Which expert kernels moe_experts / moe_forward use (process-wide). */
+/* Which expert kernels run (per call through moe_exec_cfg, or the process-wide
+ * default of moe_set_dispatch). */
 typedef enum {
     MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM, except affine
                               4-bit experts at <= 8 routed pairs per expert on average
@@ -156,6 +159,18 @@ typedef struct {
 
 #define MOE_TILE_M 128
 
+/* Per-call execution choices.  Every entry point that takes a
+ * `const moe_exec_cfg*` reads it once per call; NULL means the process-wide
+ * defaults set by moe_set_dispatch / moe_set_combine.  Two callers in one
+ * process that pass their own cfg never affect each other's kernels or
+ * workspace sizes.  MOE_ERR_UNSUPPORTED for a value outside the enums.
+ *   dispatch: moe_dispatch (which expert kernels run)
+ *   combine:  moe_combine  (atomic or slot-ordered combine; see moe_set_combine) */
+typedef struct {
+    int32_t dispatch;
+    int32_t combine;
+} moe_exec_cfg;
+
 /* Byte offsets of the regions inside the workspace (for inspection/tests). */
 typedef struct {
     size_t y_acc;   /* fp32 (T, H): the unscaled routed sum; (P, H) weighted slot outputs
@@ -171,6 +186,11 @@ typedef struct {
  * regions; ws itself must be 256-byte aligned. */
 MOE_API size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt);
 MOE_API moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* out);
+/* The same for the combine mode of `exec` (NULL = the process-wide default);
+ * 0 / MOE_ERR_UNSUPPORTED for an invalid exec. */
+MOE_API size_t moe_workspace_bytes_ex(const moe_dims* d, int32_t fmt, const moe_exec_cfg* exec);
+MOE_API moe_status moe_workspace_layout_ex(const moe_dims* d, int32_t fmt, const moe_exec_cfg* exec,
+                                           moe_ws_layout* out);
 
 /* Router.  Exactly one of x (bf16 (T, H)) or logits (fp32 (T, E)) is given;
  * with x, w_router (fp32 (E, H)) is required and the logits are computed in
@@ -197,6 +217,25 @@ MOE_API moe_status moe_experts(const void* x, const moe_plan_t* plan, const floa
                        const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
                        void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* moe_experts with a per-call exec cfg, a skipped plan expert and a shared
+ * expert's output.
+ *   skip_expert = -1: as moe_experts.
+ *   skip_expert = s in [0, E): the pairs the plan routes to plan expert s are
+ *     computed nowhere and left out of the combine, and the rows they own
+ *     (their h rows, and their slot rows under the ordered combine) are not
+ *     written.  This is the 9-slot plan of TensorFold issue #548 ("Paths your
+ *     experts test does not reach", the skip-a-slot row): top-8 plus the
+ *     shared expert's id E over E + 1 plan experts, with id E skipped, gives
+ *     the bytes of the 8-slot block.  Here d->E counts the plan experts; W
+ *     holds d->E - 1 experts when s == d->E - 1 (the shared id has no routed
+ *     weights), else d->E.  MOE_ERR_SHAPE for s outside [-1, E) or s >= 0 with E == 1.
+ *   y_shared: fp32 (T, H) or NULL, added after the routed scale as in
+ *     moe_forward_ex. */
+MOE_API moe_status moe_experts_ex(const void* x, const moe_plan_t* plan, const float* topk_w,
+                                  const moe_dims* d, const moe_experts_w* W, const moe_exec_cfg* exec,
+                                  int32_t skip_expert, const float* y_shared, float out_scale, void* y,
+                                  void* ws, size_t ws_bytes, moe_stream_t stream);
+
 /* route -> plan -> experts -> combine in one call (same arguments as the three
  * calls; logits may be NULL to route from x). */
 MOE_API moe_status moe_forward(const void* x, const float* logits, const float* w_router,
@@ -212,7 +251,9 @@ MOE_API moe_status moe_forward(const void* x, const float* logits, const float* 
  * (T, H) shared-expert output (from moe_shared_expert) or NULL: the output is
  * then y = bf16_rn(out_scale * routed sum + y_shared) -- the routed scale
  * multiplies the routed sum before the shared term is added, which itself is
- * not scaled (vllm.cpp PR #684, "The finding that justifies the row"). */
+ * not scaled (vllm.cpp PR #684, "The finding that justifies the row").
+ * moe_forward_ex's exec (NULL = the process-wide defaults) picks its expert
+ * kernels and combine mode for this call. */
 MOE_API moe_status moe_route_ex(const void* x, const float* logits, const float* w_router,
                                 const float* expert_bias, const moe_dims* d, float eps, float scale,
                                 const moe_router_cfg* cfg, int32_t* topk_idx, float* topk_w,
@@ -220,6 +261,7 @@ MOE_API moe_status moe_route_ex(const void* x, const float* logits, const float*
 MOE_API moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
                                   const float* expert_bias, const moe_dims* d, float eps,
                                   float router_scale, float out_scale, const moe_router_cfg* cfg,
+                                  const moe_exec_cfg* exec,
                                   const float* y_shared, const moe_experts_w* W, int32_t* topk_idx,
                                   float* topk_w,
                                   const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
@@ -235,6 +277,10 @@ MOE_API moe_status moe_forward_ex(const void* x, const float* logits, const floa
  * over a one-expert identity plan.  MOE_ERR_SHAPE unless E == 1 and k == 1. */
 MOE_API moe_status moe_shared_expert(const void* x, const moe_experts_w* Ws, const moe_dims* d,
                                      float* y_shared, void* ws, size_t ws_bytes, moe_stream_t stream);
+/* moe_shared_expert with a per-call exec cfg (NULL = the process-wide defaults). */
+MOE_API moe_status moe_shared_expert_ex(const void* x, const moe_experts_w* Ws, const moe_dims* d,
+                                        const moe_exec_cfg* exec, float* y_shared, void* ws,
+                                        size_t ws_bytes, moe_stream_t stream);
 
 /* moe_forward with HOST buffers for the token rows: x_host (T, H) bf16 is
  * copied to x_dev, the block runs, and y_dev is copied back to y_host (T, H)
@@ -292,10 +338,12 @@ MOE_API moe_status moe_forward_static(const void* x, const float* logits, const 
                                       int32_t* topk_idx, float* topk_w, const moe_plan_t* plan,
                                       void* y, moe_stream_t stream);
 
-/* Process-wide choice of expert kernels (moe_dispatch); returns the old one. */
+/* Process-wide default choice of expert kernels (moe_dispatch), used by calls
+ * given no moe_exec_cfg; returns the old one. */
 MOE_API int32_t moe_set_dispatch(int32_t mode);
 
-/* How the weighted expert outputs of a token are combined (process-wide).
+/* How the weighted expert outputs of a token are combined: the process-wide
+ * default, used by calls given no moe_exec_cfg.
  *   MOE_COMBINE_ATOMIC  (default): the down projection adds w_j * o_j into the
  *     fp32 accumulator y_acc (T, H) with atomic reductions; the order of the
  *     k additions, and so the last bits of y, can vary from run to run.
@@ -305,10 +353,22 @@ MOE_API int32_t moe_set_dispatch(int32_t mode);
  *     bitwise reproducible, and for bf16 experts a token's y does not depend
  *     on the other tokens of the batch (the router already has a fixed
  *     summation order).  The workspace is larger (P * H * 4 bytes for that
- *     region): query moe_workspace_bytes after setting the mode.  Not used by
+ *     region): query moe_workspace_bytes after setting the mode, or pass the mode
+ *     per call through moe_exec_cfg and moe_workspace_bytes_ex.  Not used by
  *     moe_forward_static. */
 typedef enum { MOE_COMBINE_ATOMIC = 0, MOE_COMBINE_ORDERED = 1 } moe_combine;
 MOE_API int32_t moe_set_combine(int32_t mode);
+
+/* Failure-detection check (the pages have no counterpart; this exercises the
+ * library's own stall detection).  Every mbarrier wait of the tcgen05
+ * pipelines is bounded: when its poll limit runs out the kernel writes device
+ * error code 2, drains what it issued, frees its TMEM and returns.  This call
+ * launches one single-warp kernel that runs that same bounded wait, with a
+ * limit of `polls` polls (1 <= polls <= 2^20), on an mbarrier nothing arrives
+ * on -- no TMA, no TMEM, no other work -- so the wait expires, code 2 is
+ * written and the kernel returns.  moe_device_error then reports code 2 and
+ * the context stays usable.  MOE_ERR_SHAPE for polls out of range. */
+MOE_API moe_status moe_wait_bound_check(uint32_t polls, moe_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device.  *code = 0 when no kernel reported an error.  Codes:

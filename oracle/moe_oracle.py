@@ -33,6 +33,11 @@ What it computes, and where each step is stated:
   affine-4   TensorFold pull #1492, "What": MLX affine 4-bit experts,
              dequantised exactly in float64 as in its "Verification" section
              (the float64 reference dequantises the MLX weights exactly).
+  nvfp4      TensorFold issue #548: NVFP4 experts read as stored in the
+             ModelOpt layout, "weight uint8 [N, K/2], weight_scale e4m3
+             [N, K/16], weight_scale_2 as the global scale", W4A16; its
+             skip/down_scale rows name the down projection's own global scale.
+             Dequantised exactly in float64: w = e2m1(code) * e4m3(scale) * g.
 
 Readings where the pages are silent:
   * the bias is added to the sigmoid score, c = s + b, for selection only;
@@ -40,7 +45,11 @@ Readings where the pages are silent:
     every number, -0.0 == +0.0; the k picks are returned in rank order;
   * an all-NaN row picks experts 0..k-1; its weights, and so its output row,
     are NaN;
-  * relu^2 keeps NaN (u > 0 ? u : (NaN ? u : 0)) and then squares.
+  * relu^2 keeps NaN (u > 0 ? u : (NaN ? u : 0)) and then squares;
+  * NVFP4: the low nibble of a code byte is the lower k; e2m1 is 1 sign,
+    2 exponent (bias 1) and 1 mantissa bit with no inf/NaN; the block scale is
+    e4m3 "fn" (bias 7, no infinities, 0x7F/0xFF NaN); each expert has one
+    fp32 global scale for W1 (gate and up together) and one for W2.
 
 Router and activation variants (TensorFold issue #548: the table of pieces
 each model family builds lists "routers (softmax, sigmoid + bias)"; its
@@ -74,7 +83,7 @@ import numpy as np
 
 __all__ = [
     "bf16_to_f64", "router_logits", "sigmoid", "select_topk", "select_topk_bruteforce",
-    "route", "tie_margins", "plan", "dequant_affine4", "silu", "swiglu", "relu2", "softmax",
+    "route", "tie_margins", "plan", "dequant_affine4", "e2m1_value", "e4m3_value", "dequant_nvfp4", "silu", "swiglu", "relu2", "softmax",
     "clamp_swiglu_inputs",
     "expert_outputs", "combine", "moe_block", "moe_block_all_experts", "shared_expert", "experts_block",
     "BM",
@@ -241,6 +250,40 @@ def dequant_affine4(q_words: np.ndarray, scale_bits: np.ndarray, bias_bits: np.n
     return s * codes + b
 
 
+def e2m1_value(code) -> np.ndarray:
+    """Value of 4-bit e2m1 codes: bit 3 sign, bits 2-1 exponent e, bit 0
+    mantissa m; e == 0 is subnormal (m * 0.5), else 2^(e - 1) * (1 + m / 2)."""
+    c = np.asarray(code).astype(np.int64) & 0xF
+    e = (c >> 1) & 3
+    m = (c & 1).astype(np.float64)
+    mag = np.where(e == 0, m * 0.5, np.ldexp(1.0 + m / 2.0, e - 1))
+    return np.where(c & 8, -mag, mag)
+
+
+def e4m3_value(byte) -> np.ndarray:
+    """Value of e4m3 ("fn") bytes: bit 7 sign, bits 6-3 exponent e (bias 7),
+    bits 2-0 mantissa m; e == 0 is subnormal (m / 8 * 2^-6); exponent 15 with
+    mantissa 7 is NaN (no infinities)."""
+    b = np.asarray(byte).astype(np.int64) & 0xFF
+    e = (b >> 3) & 0xF
+    m = (b & 7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(m / 8.0, -6), np.ldexp(1.0 + m / 8.0, e - 7))
+    mag = np.where((e == 15) & (b & 7 == 7), np.nan, mag)
+    return np.where(b & 0x80, -mag, mag)
+
+
+def dequant_nvfp4(codes: np.ndarray, scales: np.ndarray, global_scale: float) -> np.ndarray:
+    """NVFP4 (ModelOpt layout) to float64: w[n, k] = e2m1(q[n, k]) *
+    e4m3(scale[n, k // 16]) * global_scale.
+
+    codes (..., N, K/2) uint8 with the lower k in the low nibble; scales
+    (..., N, K/16) uint8 e4m3 bytes; global_scale the fp32 weight_scale_2."""
+    p = np.asarray(codes, dtype=np.uint8)
+    q = np.stack([p & 0xF, p >> 4], axis=-1).reshape(*p.shape[:-1], p.shape[-1] * 2)
+    s = np.repeat(e4m3_value(scales), 16, axis=-1)
+    return e2m1_value(q) * s * float(np.float32(global_scale))
+
+
 def silu(g):
     with np.errstate(over="ignore", invalid="ignore"):
         return g / (1.0 + np.exp(-g))
@@ -261,6 +304,9 @@ def _expert_w(inp, which: str, e: int) -> np.ndarray:
     """float64 (N, K) weight of expert e (which = 'w1' or 'w2')."""
     if inp.wl.fmt == "bf16":
         return bf16_to_f64(getattr(inp, which + "_bits")[e])
+    if inp.wl.fmt == "nvfp4":
+        return dequant_nvfp4(getattr(inp, which + "_q")[e], getattr(inp, which + "_scale")[e],
+                             getattr(inp, which + "_global")[e])
     return dequant_affine4(getattr(inp, which + "_q")[e], getattr(inp, which + "_scale")[e],
                            getattr(inp, which + "_bias")[e])
 
@@ -311,6 +357,8 @@ def _shared_w(inp, which: str) -> np.ndarray:
     sh = inp.shared
     if inp.wl.fmt == "bf16":
         return bf16_to_f64(sh[which + "_bits"][0])
+    if inp.wl.fmt == "nvfp4":
+        return dequant_nvfp4(sh[which + "_q"][0], sh[which + "_scale"][0], sh[which + "_global"][0])
     return dequant_affine4(sh[which + "_q"][0], sh[which + "_scale"][0], sh[which + "_bias"][0])
 
 

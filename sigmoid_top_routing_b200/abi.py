@@ -41,6 +41,10 @@ class moe_router_cfg(ctypes.Structure):
     _fields_ = [("score", c_int32), ("norm_topk", c_int32)]
 
 
+class moe_exec_cfg(ctypes.Structure):
+    _fields_ = [("dispatch", c_int32), ("combine", c_int32)]
+
+
 class moe_plan_t(ctypes.Structure):
     _fields_ = [("counts", c_void_p), ("offsets", c_void_p), ("perm", c_void_p), ("inv", c_void_p),
                 ("tiles", c_void_p)]
@@ -55,6 +59,9 @@ class moe_ws_layout(ctypes.Structure):
 PROTOTYPES = {
     "moe_workspace_bytes": (c_size_t, [POINTER(moe_dims), c_int32]),
     "moe_workspace_layout": (c_int32, [POINTER(moe_dims), c_int32, POINTER(moe_ws_layout)]),
+    "moe_workspace_bytes_ex": (c_size_t, [POINTER(moe_dims), c_int32, POINTER(moe_exec_cfg)]),
+    "moe_workspace_layout_ex": (c_int32, [POINTER(moe_dims), c_int32, POINTER(moe_exec_cfg),
+                                          POINTER(moe_ws_layout)]),
     "moe_route": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
                             c_void_p, c_void_p, c_void_p]),
     "moe_plan": (c_int32, [c_void_p, POINTER(moe_dims), POINTER(moe_plan_t), c_void_p, c_size_t, c_void_p]),
@@ -63,13 +70,19 @@ PROTOTYPES = {
     "moe_forward": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
                               c_float, POINTER(moe_experts_w), c_void_p, c_void_p, POINTER(moe_plan_t),
                               c_void_p, c_void_p, c_size_t, c_void_p]),
+    "moe_experts_ex": (c_int32, [c_void_p, POINTER(moe_plan_t), c_void_p, POINTER(moe_dims),
+                                 POINTER(moe_experts_w), POINTER(moe_exec_cfg), c_int32, c_void_p, c_float,
+                                 c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_route_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
                                POINTER(moe_router_cfg), c_void_p, c_void_p, c_void_p]),
     "moe_forward_ex": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float, c_float,
-                                 c_float, POINTER(moe_router_cfg), c_void_p, POINTER(moe_experts_w), c_void_p,
+                                 c_float, POINTER(moe_router_cfg), POINTER(moe_exec_cfg), c_void_p,
+                                 POINTER(moe_experts_w), c_void_p,
                                  c_void_p, POINTER(moe_plan_t), c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_shared_expert": (c_int32, [c_void_p, POINTER(moe_experts_w), POINTER(moe_dims), c_void_p, c_void_p,
                                     c_size_t, c_void_p]),
+    "moe_shared_expert_ex": (c_int32, [c_void_p, POINTER(moe_experts_w), POINTER(moe_dims),
+                                       POINTER(moe_exec_cfg), c_void_p, c_void_p, c_size_t, c_void_p]),
     "moe_forward_host": (c_int32, [c_void_p, c_void_p, c_void_p, c_void_p, POINTER(moe_dims), c_float,
                                    c_float, c_float, POINTER(moe_experts_w), c_void_p, c_void_p,
                                    POINTER(moe_plan_t), c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -81,6 +94,7 @@ PROTOTYPES = {
     "moe_set_dispatch": (c_int32, [c_int32]),
     "moe_set_combine": (c_int32, [c_int32]),
     "moe_device_error": (c_int32, [POINTER(c_int32), c_void_p]),
+    "moe_wait_bound_check": (c_int32, [ctypes.c_uint32, c_void_p]),
     "moe_last_error": (c_char_p, []),
     "moe_version": (c_char_p, []),
 }

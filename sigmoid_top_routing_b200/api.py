@@ -20,7 +20,7 @@ __all__ = [
     "moe_experts", "moe_forward", "moe_forward_host", "moe_shared_expert", "moe_set_dispatch", "moe_set_combine",
     "moe_device_error",
     "moe_last_error", "moe_version", "new_plan", "new_workspace", "dims", "moe_profile_hook",
-    "moe_last_launch_count",
+    "moe_last_launch_count", "exec_cfg", "moe_experts_ex",
 ]
 
 
@@ -67,6 +67,20 @@ def router_cfg(score: str = "sigmoid", norm_topk: bool = True) -> abi.moe_router
                               1 if norm_topk else 0)
 
 
+def exec_cfg(dispatch: Optional[int] = None, combine: Optional[int] = None) -> Optional[abi.moe_exec_cfg]:
+    """A per-call execution choice, or None (the library's process-wide
+    defaults) when neither is given; a missing one of the two takes the
+    library's default value (AUTO dispatch, atomic combine)."""
+    if dispatch is None and combine is None:
+        return None
+    return abi.moe_exec_cfg(abi.MOE_DISPATCH_AUTO if dispatch is None else dispatch,
+                            abi.MOE_COMBINE_ATOMIC if combine is None else combine)
+
+
+def _ref(c):
+    return None if c is None else ctypes.byref(c)
+
+
 @dataclasses.dataclass
 class Plan:
     counts: torch.Tensor   # [E] int32
@@ -86,18 +100,21 @@ def new_plan(T: int, E: int, k: int, device="cuda") -> Plan:
     return Plan(z(E), z(E + 1), z(P), z(P), z(E + 1))
 
 
-def moe_workspace_bytes(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16) -> int:
-    return int(load().moe_workspace_bytes(ctypes.byref(d), fmt))
+def moe_workspace_bytes(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16, *, dispatch=None, combine=None) -> int:
+    return int(load().moe_workspace_bytes_ex(ctypes.byref(d), fmt, _ref(exec_cfg(dispatch, combine))))
 
 
-def moe_workspace_layout(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16) -> abi.moe_ws_layout:
+def moe_workspace_layout(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16, *, dispatch=None,
+                         combine=None) -> abi.moe_ws_layout:
     out = abi.moe_ws_layout()
-    check(load().moe_workspace_layout(ctypes.byref(d), fmt, ctypes.byref(out)), "moe_workspace_layout")
+    check(load().moe_workspace_layout_ex(ctypes.byref(d), fmt, _ref(exec_cfg(dispatch, combine)),
+                                         ctypes.byref(out)), "moe_workspace_layout")
     return out
 
 
-def new_workspace(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16, device="cuda") -> torch.Tensor:
-    n = moe_workspace_bytes(d, fmt)
+def new_workspace(d: abi.moe_dims, fmt: int = abi.MOE_W_BF16, device="cuda", *, dispatch=None,
+                  combine=None) -> torch.Tensor:
+    n = moe_workspace_bytes(d, fmt, dispatch=dispatch, combine=combine)
     if n == 0:
         raise ValueError("invalid sizes for a workspace")
     return torch.empty(n, dtype=torch.uint8, device=device)
@@ -135,22 +152,30 @@ def moe_plan(topk_idx, *, E: int, H: int = 64, I: int = 64, plan: Optional[Plan]
 
 
 def moe_experts(x, plan: Plan, topk_w, W: ExpertWeights, *, E: int, I: int, out_scale: float = 1.0, y=None,
-                ws=None, stream=None):
+                ws=None, stream=None, skip: int = -1, y_shared=None, dispatch=None, combine=None):
+    """Grouped experts + combine over a plan of E plan experts; ``skip`` >= 0
+    names a plan expert whose pairs are computed nowhere and left out (W then
+    holds E - 1 experts when skip == E - 1)."""
     T, H = x.shape
     k = topk_w.shape[1]
     d = abi.moe_dims(T, H, E, k, I)
     y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=x.device)
-    ws = ws if ws is not None else new_workspace(d, W.fmt, x.device)
+    ex = exec_cfg(dispatch, combine)
+    ws = ws if ws is not None else new_workspace(d, W.fmt, x.device, dispatch=dispatch, combine=combine)
     cp, cw = plan.c_struct(), W.c_struct()
-    check(load().moe_experts(_ptr(x), ctypes.byref(cp), _ptr(topk_w), ctypes.byref(d), ctypes.byref(cw),
-                             out_scale, _ptr(y), _ptr(ws), ws.numel(), _stream(stream)), "moe_experts")
+    check(load().moe_experts_ex(_ptr(x), ctypes.byref(cp), _ptr(topk_w), ctypes.byref(d), ctypes.byref(cw),
+                                _ref(ex), skip, _ptr(y_shared), out_scale, _ptr(y), _ptr(ws), ws.numel(),
+                                _stream(stream)), "moe_experts")
     return y
+
+
+moe_experts_ex = moe_experts
 
 
 def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int, k: int, I: int,
                 logits=None, eps: float = 1e-6, router_scale: float = 1.0, out_scale: float = 1.0,
                 topk_idx=None, topk_w=None, plan: Optional[Plan] = None, y=None, ws=None, stream=None,
-                score: str = "sigmoid", norm_topk: bool = True, y_shared=None):
+                score: str = "sigmoid", norm_topk: bool = True, y_shared=None, dispatch=None, combine=None):
     T, H = x.shape
     d = abi.moe_dims(T, H, E, k, I)
     dev = x.device
@@ -158,24 +183,28 @@ def moe_forward(x, W: ExpertWeights, w_router=None, expert_bias=None, *, E: int,
     topk_w = topk_w if topk_w is not None else torch.empty((T, k), dtype=torch.float32, device=dev)
     plan = plan or new_plan(T, E, k, dev)
     y = y if y is not None else torch.empty((T, H), dtype=torch.bfloat16, device=dev)
-    ws = ws if ws is not None else new_workspace(d, W.fmt, dev)
+    ex = exec_cfg(dispatch, combine)
+    ws = ws if ws is not None else new_workspace(d, W.fmt, dev, dispatch=dispatch, combine=combine)
     cp, cw, rc = plan.c_struct(), W.c_struct(), router_cfg(score, norm_topk)
     check(load().moe_forward_ex(_ptr(x), _ptr(logits), _ptr(w_router), _ptr(expert_bias), ctypes.byref(d), eps,
-                                router_scale, out_scale, ctypes.byref(rc), _ptr(y_shared), ctypes.byref(cw),
+                                router_scale, out_scale, ctypes.byref(rc), _ref(ex), _ptr(y_shared),
+                                ctypes.byref(cw),
                                 _ptr(topk_idx), _ptr(topk_w), ctypes.byref(cp), _ptr(y), _ptr(ws), ws.numel(),
                                 _stream(stream)), "moe_forward")
     return y, topk_idx, topk_w, plan
 
 
-def moe_shared_expert(x, Ws: ExpertWeights, *, I: int, y_shared=None, ws=None, stream=None):
+def moe_shared_expert(x, Ws: ExpertWeights, *, I: int, y_shared=None, ws=None, stream=None, dispatch=None,
+                      combine=None):
     """fp32 (T, H) output of the shared expert (one expert, weight 1, on every token)."""
     T, H = x.shape
     d = abi.moe_dims(T, H, 1, 1, I)
     y_shared = y_shared if y_shared is not None else torch.empty((T, H), dtype=torch.float32, device=x.device)
-    ws = ws if ws is not None else new_workspace(d, Ws.fmt, x.device)
+    ex = exec_cfg(dispatch, combine)
+    ws = ws if ws is not None else new_workspace(d, Ws.fmt, x.device, dispatch=dispatch, combine=combine)
     cw = Ws.c_struct()
-    check(load().moe_shared_expert(_ptr(x), ctypes.byref(cw), ctypes.byref(d), _ptr(y_shared), _ptr(ws),
-                                   ws.numel(), _stream(stream)), "moe_shared_expert")
+    check(load().moe_shared_expert_ex(_ptr(x), ctypes.byref(cw), ctypes.byref(d), _ref(ex), _ptr(y_shared),
+                                      _ptr(ws), ws.numel(), _stream(stream)), "moe_shared_expert")
     return y_shared
 
 

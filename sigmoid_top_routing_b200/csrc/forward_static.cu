@@ -159,6 +159,8 @@ extern "C" moe_status moe_forward_static(const void* x, const float* logits, con
     a.T = d->T;
     a.H = d->H;
     a.E = d->E;
+    a.E_w = d->E;
+    a.skip = -1;              // every plan expert has weights and is computed
     a.k = d->k;
     a.I = d->I;
     a.act = W->act;

@@ -72,6 +72,9 @@ struct GemmParams {
     const uint16_t* wscale;  // affine 4-bit: (E, rows_per_expert, K/64) bf16 scales
     const uint16_t* wbias;   //                and biases
     float swiglu_limit;      // up SwiGLU: clamp of the gate (above) and up (both sides); 0 off
+    int skip;                // plan expert given no tiles (its pairs are computed nowhere), or -1
+    int E_w;                 // experts the weight tensor holds
+    uint32_t wait_limit;     // polls of every bounded pipeline wait (sm100::kWaitLimit)
     int* err;
 };
 
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     // right before the first load of h.
     if (MODE != kDown) pdl_wait();
     for (int i = threadIdx.x; i < g.E; i += blockDim.x) {
-        s_cnt[i] = __ldcg(g.counts + i);
+        s_cnt[i] = i == g.skip ? 0 : __ldcg(g.counts + i);   // a skipped expert gets no tiles
         s_off[i] = __ldcg(g.offsets + i);
     }
     __syncthreads();
@@ -354,7 +357,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     continue;
                 }
                 // all 32 lanes wait on the same phase; the decision is made warp-uniform
-                const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort);
+                const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort, g.wait_limit);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 if (lane == 0) {
                     const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
@@ -389,7 +392,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         }
         // wait (bounded) for every fill this warp issued to land before the CTA can exit
         for (int q = 0; q < STAGES; ++q)
-            if (issued_mask >> q & 1u) mbar_wait(&full[q], issued_par >> q & 1u, nullptr);
+            if (issued_mask >> q & 1u) mbar_wait(&full[q], issued_par >> q & 1u, nullptr, g.wait_limit);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -401,12 +404,12 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
                 const int buf = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
-                if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort)) { ok = false; break; }
+                if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort, g.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * (kDual ? 2 * BN : BN);
                 const uint32_t idesc = idesc_bf16(128, tl.n);
                 for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
-                    if (!mbar_wait(&full[s], ph, s_abort)) { ok = false; break; }
+                    if (!mbar_wait(&full[s], ph, s_abort, g.wait_limit)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t ad = sdesc_sw128(smem_u32(sA + size_t(s) * kAStage));
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             }
             // all MMAs issued by this thread complete before TMEM is freed
             umma_commit(drain);
-            mbar_wait(drain, 0, nullptr);
+            mbar_wait(drain, 0, nullptr, g.wait_limit);
         }
         __syncwarp();
     } else if (WFMT && warp >= 6) {   // warps 6..13
@@ -443,7 +446,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         const int r = kDual ? dt : (dt >> 1);
         const int cbeg = kDual ? 0 : (dt & 1) * 4;
         const int halfr = kDual ? 128 : 64;                // SwiGLU: rows of the gate half
-        const size_t nrows = (size_t)g.E * g.rows_per_expert;
+        const size_t nrows = (size_t)g.E_w * g.rows_per_expert;
         const int G = g.K / 64;
         uint32_t* s_sb = reinterpret_cast<uint32_t*>(sm + L::kSB);
         auto grow = [&](const Tile& tl) -> size_t {      // global weight row of A row r
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 const uint16_t bi = inb ? uint16_t(odd ? bw >> 16 : bw & 0xFFFFu) : uint16_t(0);
                 issue(slot);                                  // refill the slot kSBDepth stages ahead
                 if (++slot == kSBDepth) slot = 0;
-                if (!mbar_wait(&cfull[s], ph, s_abort)) { ok = false; break; }
+                if (!mbar_wait(&cfull[s], ph, s_abort, g.wait_limit)) { ok = false; break; }
                 const uint32_t* crow = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage) + r * 8 + cbeg;
                 uint32_t cw[kCPT];
 #pragma unroll
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 named_bar(1, 128);
             }
             if (!dead) {
-                const bool ok = mbar_wait(&tfull[buf], aph, s_abort);
+                const bool ok = mbar_wait(&tfull[buf], aph, s_abort, g.wait_limit);
                 if (__any_sync(0xffffffffu, !ok)) {     // warp-uniform: tcgen05.ld is warp-collective
                     if (lane == 0) report_error(g.err, kErrWaitExpired);
                     *s_abort = 1;
@@ -690,9 +693,9 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     const uint32_t b_box = BN < 64 ? 16 : 64;
     cudaError_t e;
     if (WFMT)   // 8 code words (64 codes) of one k-block per row
-        e = make_tmap_u32(&tA, wbase, (uint64_t)g.K / 8, (uint64_t)g.E * g.rows_per_expert, 8, a_box);
+        e = make_tmap_u32(&tA, wbase, (uint64_t)g.K / 8, (uint64_t)g.E_w * g.rows_per_expert, 8, a_box);
     else
-        e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E * g.rows_per_expert, kBK, a_box);
+        e = make_tmap(&tA, wbase, (uint64_t)g.K, (uint64_t)g.E_w * g.rows_per_expert, kBK, a_box);
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
         e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, b_box);
@@ -732,6 +735,9 @@ GemmParams params(const ExpertArgs& a, bool up) {
     g.k = a.k;
     g.H = a.H;
     g.I = a.I;
+    g.skip = a.skip;
+    g.E_w = a.E_w;
+    g.wait_limit = kWaitLimit;
     g.err = a.err;
     if (up) {
         g.K = a.H;

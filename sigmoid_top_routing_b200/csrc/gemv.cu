@@ -27,14 +27,15 @@ constexpr int kWarps = 8;
 constexpr int kTokGroup = 8;          // tokens whose partial sums a warp keeps at once
 constexpr int kChunksPerLane = 8;     // 16-byte chunks of a row a lane holds per pass
 
-// Active experts (count > 0) compacted in id order into s_act; returns how many.
-MOE_DEV int build_active(const int32_t* counts, int E, int* s_act, int* s_n) {
+// Active experts (count > 0, not the skipped one) compacted in id order into
+// s_act; returns how many.
+MOE_DEV int build_active(const int32_t* counts, int E, int skip, int* s_act, int* s_n) {
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         int base = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
-            const bool on = e < E && counts[e] > 0;
+            const bool on = e < E && e != skip && counts[e] > 0;
             const unsigned m = __ballot_sync(0xffffffffu, on);
             if (on) s_act[base + __popc(m & ((1u << lane) - 1u))] = e;
             base += __popc(m);
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_gemv_up(ExpertArgs a) {
     __shared__ int s_n;
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_act = build_active(a.counts, a.E, s_act, &s_n);
+    const int n_act = build_active(a.counts, a.E, a.skip, s_act, &s_n);
     const int I = a.I, H = a.H;
     const int n1 = ACT == 0 ? 2 * I : I;
     const int upe = (I + kWarps - 1) / kWarps;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) k_gemv_down(ExpertArgs a) {
     __shared__ int s_n;
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_act = build_active(a.counts, a.E, s_act, &s_n);
+    const int n_act = build_active(a.counts, a.E, a.skip, s_act, &s_n);
     const int I = a.I, H = a.H;
     const int upe = (H + kWarps - 1) / kWarps;
     const long long total = (long long)n_act * upe;
@@ -211,17 +212,22 @@ __global__ void __launch_bounds__(256) k_finalize(ExpertArgs a) {
 }
 
 // Ordered combine: y[t] = bf16_rn(out_scale * (sum over j = 0..k-1, in that
-// order, of the slot row inv[t * k + j])); the rows already carry w_j.
+// order, of the slot row inv[t * k + j])); the rows already carry w_j.  Slots
+// of the skipped plan expert (positions offsets[skip] .. offsets[skip + 1])
+// hold nothing and are left out.
 __global__ void __launch_bounds__(256) k_finalize_ordered(ExpertArgs a) {
     pdl_wait();
     const size_t n4 = (size_t)a.T * a.H / 4;
     const int h4 = a.H / 4;
     const float sc = a.out_scale;
+    const int skip_lo = a.skip >= 0 ? a.offsets[a.skip] : 0;
+    const int skip_hi = a.skip >= 0 ? a.offsets[a.skip + 1] : 0;
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const int t = (int)(i / h4), c = (int)(i - (size_t)t * h4);
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int j = 0; j < a.k; ++j) {
             const int slot = a.inv[(size_t)t * a.k + j];
+            if (slot >= skip_lo && slot < skip_hi) continue;
             const float4 v = __ldcg(reinterpret_cast<const float4*>(a.y_acc + (size_t)slot * a.H) + c);
             s.x += v.x;
             s.y += v.y;

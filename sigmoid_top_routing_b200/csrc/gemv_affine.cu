@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kA4Warps * 32, 4) k_gemv_a4(ExpertArgs a) {
         int run = 0;
         for (int e0 = 0; e0 < a.E; e0 += 32) {
             const int e = e0 + lane;
-            const int nu = e < a.E ? (a.counts[e] + kA4Tok - 1) / kA4Tok * RQ : 0;
+            const int nu = (e < a.E && e != a.skip) ? (a.counts[e] + kA4Tok - 1) / kA4Tok * RQ : 0;
             int v = nu;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {

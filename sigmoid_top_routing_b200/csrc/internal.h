@@ -47,7 +47,9 @@ struct ExpertArgs {
     const int32_t* perm;
     const int32_t* inv;      // pair t * k + j -> plan slot (ordered combine)
     const int32_t* tiles;
-    int T, H, E, k, I;
+    int T, H, E, k, I;       // E: plan experts
+    int E_w;                 // experts the weight tensors hold (E, or E - 1 when the last is skipped)
+    int skip;                // plan expert whose pairs are computed nowhere and left out, or -1
     int act;                 // 0 swiglu, 1 relu2
     int fmt;                 // 0 bf16, 1 affine4
     float swiglu_limit;      // > 0: g = min(g, L), u = clamp(u, -L, L) before silu(g) * u

@@ -49,11 +49,6 @@ std::mutex g_dispatch_mu;
 int g_dispatch = MOE_DISPATCH_AUTO;
 int g_combine = MOE_COMBINE_ATOMIC;   // guarded by g_dispatch_mu
 
-bool combine_ordered() {
-    std::lock_guard<std::mutex> lock(g_dispatch_mu);
-    return g_combine == MOE_COMBINE_ORDERED;
-}
-
 moe_status fail(moe_status st, const char* fmt, ...) {
     char buf[512];
     va_list ap;
@@ -91,6 +86,29 @@ moe_status check_fmt(int32_t fmt) {
     return MOE_OK;
 }
 
+// A call's execution choices, read once per call.
+struct Exec {
+    int dispatch;            // moe_dispatch
+    bool ordered;            // slot-ordered combine
+};
+
+// The call's cfg, or the process-wide defaults when it passes none.
+moe_status resolve_exec(const moe_exec_cfg* cfg, Exec* x) {
+    if (!cfg) {
+        std::lock_guard<std::mutex> lock(g_dispatch_mu);
+        x->dispatch = g_dispatch;
+        x->ordered = g_combine == MOE_COMBINE_ORDERED;
+        return MOE_OK;
+    }
+    if (cfg->dispatch != MOE_DISPATCH_AUTO && cfg->dispatch != MOE_DISPATCH_GEMV && cfg->dispatch != MOE_DISPATCH_GEMM)
+        return fail(MOE_ERR_UNSUPPORTED, "exec dispatch %d", cfg->dispatch);
+    if (cfg->combine != MOE_COMBINE_ATOMIC && cfg->combine != MOE_COMBINE_ORDERED)
+        return fail(MOE_ERR_UNSUPPORTED, "exec combine %d", cfg->combine);
+    x->dispatch = cfg->dispatch;
+    x->ordered = cfg->combine == MOE_COMBINE_ORDERED;
+    return MOE_OK;
+}
+
 // ordered: the combine mode the call runs with (read once per call)
 void layout(const moe_dims* d, moe_ws_layout* L, bool ordered) {
     const size_t T = d->T, H = d->H, E = d->E, P = (size_t)d->T * d->k, I = d->I;
@@ -118,10 +136,10 @@ struct WsView {
     bool ordered;            // the combine mode of this call (read once)
 };
 
-moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, WsView* v) {
+moe_status check_ws(const moe_dims* d, void* ws, size_t ws_bytes, bool ordered, WsView* v) {
     moe_ws_layout L;
-    v->ordered = combine_ordered();
-    layout(d, &L, v->ordered);
+    v->ordered = ordered;
+    layout(d, &L, ordered);
     if (!ws) return fail(MOE_ERR_WORKSPACE, "workspace is NULL");
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_ALIGN, "workspace not 256-byte aligned");
     if (ws_bytes < L.total)
@@ -188,17 +206,11 @@ moe_status check_route_args(const void* x, const float* logits, const float* w_r
     return MOE_OK;
 }
 
-int current_dispatch() {
-    std::lock_guard<std::mutex> lock(g_dispatch_mu);
-    return g_dispatch;
-}
-
 // bf16: the tcgen05 grouped GEMM serves every token count (its token tiles
 // shrink to 32 for decode batches); the CUDA-core GEMV stays selectable.
 // Affine 4-bit: up to a few pairs per expert the register-dequant GEMV streams
 // the codes faster than the GEMM's shared-memory dequant pipeline.
-bool use_gemv(const moe_dims* d, int32_t fmt) {
-    const int mode = current_dispatch();
+bool use_gemv(const moe_dims* d, int32_t fmt, int mode) {
     if (mode != MOE_DISPATCH_AUTO) return mode == MOE_DISPATCH_GEMV;
     return fmt == MOE_W_AFFINE4_G64 && d->H <= 8192 && d->I <= 8192 &&
            (size_t)d->T * d->k <= (size_t)kAffineGemvMaxPairsPerExpert * d->E;
@@ -220,6 +232,8 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.E = d->E;
     a.k = d->k;
     a.I = d->I;
+    a.E_w = d->E;
+    a.skip = -1;
     a.act = W->act;
     a.fmt = W->fmt;
     a.swiglu_limit = W->swiglu_limit;
@@ -270,8 +284,8 @@ struct Seq {
     }
 };
 
-moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d) {
-    const bool gemv = use_gemv(d, a.fmt);
+moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d, int dispatch) {
+    const bool gemv = use_gemv(d, a.fmt, dispatch);
     cudaError_t e;
     if (!gemv) {
         // token rows in plan order for the up GEMM's TMA (part of the plan's data movement)
@@ -324,19 +338,28 @@ moe_status validate_weights(const moe_experts_w* W) { return check_weights(W); }
 
 extern "C" {
 
-size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt) {
-    if (check_dims(d) != MOE_OK || check_fmt(fmt) != MOE_OK) return 0;
+size_t moe_workspace_bytes(const moe_dims* d, int32_t fmt) { return moe_workspace_bytes_ex(d, fmt, nullptr); }
+
+size_t moe_workspace_bytes_ex(const moe_dims* d, int32_t fmt, const moe_exec_cfg* exec) {
+    Exec x;
+    if (check_dims(d) != MOE_OK || check_fmt(fmt) != MOE_OK || resolve_exec(exec, &x) != MOE_OK) return 0;
     moe_ws_layout L;
-    layout(d, &L, combine_ordered());
+    layout(d, &L, x.ordered);
     return L.total;
 }
 
 moe_status moe_workspace_layout(const moe_dims* d, int32_t fmt, moe_ws_layout* out) {
+    return moe_workspace_layout_ex(d, fmt, nullptr, out);
+}
+
+moe_status moe_workspace_layout_ex(const moe_dims* d, int32_t fmt, const moe_exec_cfg* exec, moe_ws_layout* out) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
     if ((st = check_fmt(fmt)) != MOE_OK) return st;
+    Exec x;
+    if ((st = resolve_exec(exec, &x)) != MOE_OK) return st;
     if (!out) return fail(MOE_ERR_NULL, "out is NULL");
-    layout(d, out, combine_ordered());
+    layout(d, out, x.ordered);
     return MOE_OK;
 }
 
@@ -382,8 +405,8 @@ moe_status moe_plan(const int32_t* topk_idx, const moe_dims* d, const moe_plan_t
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
     if (!topk_idx) return fail(MOE_ERR_NULL, "topk_idx is NULL");
     if ((st = check_plan(plan)) != MOE_OK) return st;
-    WsView v;
-    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    WsView v;   // the plan uses only the scratch region, placed as in the (smaller) atomic layout
+    if ((st = check_ws(d, ws, ws_bytes, false, &v)) != MOE_OK) return st;
     const PlanArgs p = make_plan_args(topk_idx, d, plan, v.plan_scratch);
     Seq q{reinterpret_cast<cudaStream_t>(stream)};
     cudaError_t e = q.stage(MOE_STAGE_PLAN, [&](int* n) { return launch_plan(p, true, q.s, n); });
@@ -395,23 +418,39 @@ moe_status moe_plan(const int32_t* topk_idx, const moe_dims* d, const moe_plan_t
 moe_status moe_experts(const void* x, const moe_plan_t* plan, const float* topk_w,
                        const moe_dims* d, const moe_experts_w* W, float out_scale, void* y,
                        void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return moe_experts_ex(x, plan, topk_w, d, W, nullptr, -1, nullptr, out_scale, y, ws, ws_bytes, stream);
+}
+
+moe_status moe_experts_ex(const void* x, const moe_plan_t* plan, const float* topk_w, const moe_dims* d,
+                          const moe_experts_w* W, const moe_exec_cfg* exec, int32_t skip_expert,
+                          const float* y_shared, float out_scale, void* y, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    if (skip_expert < -1 || skip_expert >= d->E)
+        return fail(MOE_ERR_SHAPE, "skip_expert = %d: need -1 <= skip_expert < E = %d", skip_expert, d->E);
+    if (skip_expert >= 0 && d->E < 2) return fail(MOE_ERR_SHAPE, "skip_expert needs E >= 2 plan experts");
+    Exec xc;
+    if ((st = resolve_exec(exec, &xc)) != MOE_OK) return st;
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
     if (!x || !topk_w || !y) return fail(MOE_ERR_NULL, "x, topk_w or y is NULL");
     if (!aligned16(x) || !aligned16(y)) return fail(MOE_ERR_ALIGN, "x or y not 16-byte aligned");
+    if (y_shared && !aligned16(y_shared)) return fail(MOE_ERR_ALIGN, "y_shared not 16-byte aligned");
     if ((st = check_plan(plan)) != MOE_OK) return st;
     if ((st = check_weights(W)) != MOE_OK) return st;
     WsView v;
-    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    if ((st = check_ws(d, ws, ws_bytes, xc.ordered, &v)) != MOE_OK) return st;
     Seq q{reinterpret_cast<cudaStream_t>(stream)};
-    const ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
-    if (!a.ordered) {   // the ordered combine writes every slot row: nothing to clear
+    ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
+    a.skip = skip_expert;
+    a.E_w = skip_expert == d->E - 1 ? d->E - 1 : d->E;   // the last plan expert skipped: no weights for it
+    a.y_shared = y_shared;
+    if (!a.ordered) {   // the ordered combine writes every slot row it sums: nothing to clear
         cudaError_t e = launch_zero(v.y_acc, (size_t)d->T * d->H, true, q.s);
         if (e != cudaSuccess) return cuda_fail(e, "zero y_acc");
         q.n = 1;
     }
-    if ((st = run_experts(q, a, d)) != MOE_OK) return st;
+    if ((st = run_experts(q, a, d, xc.dispatch)) != MOE_OK) return st;
     g_launches = q.n;
     return MOE_OK;
 }
@@ -422,16 +461,18 @@ moe_status moe_forward(const void* x, const float* logits, const float* w_router
                        const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
     return moe_forward_ex(x, logits, w_router, expert_bias, d, eps, router_scale, out_scale, nullptr, nullptr,
-                          W, topk_idx, topk_w, plan, y, ws, ws_bytes, stream);
+                          nullptr, W, topk_idx, topk_w, plan, y, ws, ws_bytes, stream);
 }
 
 moe_status moe_forward_ex(const void* x, const float* logits, const float* w_router,
                           const float* expert_bias, const moe_dims* d, float eps, float router_scale,
-                          float out_scale, const moe_router_cfg* cfg, const float* y_shared,
-                          const moe_experts_w* W, int32_t* topk_idx, float* topk_w, const moe_plan_t* plan,
-                          void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                          float out_scale, const moe_router_cfg* cfg, const moe_exec_cfg* exec,
+                          const float* y_shared, const moe_experts_w* W, int32_t* topk_idx, float* topk_w,
+                          const moe_plan_t* plan, void* y, void* ws, size_t ws_bytes, moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    Exec xc;
+    if ((st = resolve_exec(exec, &xc)) != MOE_OK) return st;
     if (y_shared && !aligned16(y_shared)) return fail(MOE_ERR_ALIGN, "y_shared not 16-byte aligned");
     RouteArgs r0{};
     if ((st = check_router_cfg(cfg, &r0)) != MOE_OK) return st;
@@ -444,7 +485,7 @@ moe_status moe_forward_ex(const void* x, const float* logits, const float* w_rou
     if ((st = check_plan(plan)) != MOE_OK) return st;
     if ((st = check_weights(W)) != MOE_OK) return st;
     WsView v;
-    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    if ((st = check_ws(d, ws, ws_bytes, xc.ordered, &v)) != MOE_OK) return st;
 
     RouteArgs r{};
     r.x = logits ? nullptr : static_cast<const uint16_t*>(x);
@@ -482,22 +523,29 @@ moe_status moe_forward_ex(const void* x, const float* logits, const float* w_rou
     }
     ExpertArgs a = make_expert_args(x, plan, topk_w, d, W, out_scale, y, v);
     a.y_shared = y_shared;
-    if ((st = run_experts(q, a, d)) != MOE_OK) return st;
+    if ((st = run_experts(q, a, d, xc.dispatch)) != MOE_OK) return st;
     g_launches = q.n;
     return MOE_OK;
 }
 
 moe_status moe_shared_expert(const void* x, const moe_experts_w* Ws, const moe_dims* d, float* y_shared,
                              void* ws, size_t ws_bytes, moe_stream_t stream) {
+    return moe_shared_expert_ex(x, Ws, d, nullptr, y_shared, ws, ws_bytes, stream);
+}
+
+moe_status moe_shared_expert_ex(const void* x, const moe_experts_w* Ws, const moe_dims* d, const moe_exec_cfg* exec,
+                                float* y_shared, void* ws, size_t ws_bytes, moe_stream_t stream) {
     moe_status st = check_dims(d);
     if (st != MOE_OK) return st;
+    Exec xc;
+    if ((st = resolve_exec(exec, &xc)) != MOE_OK) return st;
     if (d->E != 1 || d->k != 1) return fail(MOE_ERR_SHAPE, "the shared expert needs E == 1 and k == 1");
     if (d->T == 0) return g_launches = 0, MOE_OK;   // empty batch: nothing to do
     if (!x || !y_shared) return fail(MOE_ERR_NULL, "x or y_shared is NULL");
     if (!aligned16(x) || !aligned16(y_shared)) return fail(MOE_ERR_ALIGN, "x or y_shared not 16-byte aligned");
     if ((st = check_weights(Ws)) != MOE_OK) return st;
     WsView v;
-    if ((st = check_ws(d, ws, ws_bytes, &v)) != MOE_OK) return st;
+    if ((st = check_ws(d, ws, ws_bytes, xc.ordered, &v)) != MOE_OK) return st;
     // the identity plan and the weights of 1 live in the scratch region (at
     // E = 1 it holds >= 4224 + 32 T bytes, more than the 3 align256(4 T) + 48
     // used here); x is already in plan order, so nothing is gathered
@@ -519,7 +567,7 @@ moe_status moe_shared_expert(const void* x, const moe_experts_w* Ws, const moe_d
         if ((e = launch_zero(y_shared, T * d->H, true, q.s)) != cudaSuccess) return cuda_fail(e, "zero y_shared");
         ++q.n;
     }
-    const bool gemv = use_gemv(d, a.fmt);
+    const bool gemv = use_gemv(d, a.fmt, xc.dispatch);
     e = q.stage(MOE_STAGE_UP, [&](int*) { return gemv ? launch_gemv_up(a, true, q.s) : launch_gemm_up(a, true, q.s); });
     if (e == cudaErrorNotSupported) return fail(MOE_ERR_UNSUPPORTED, "no expert kernel for this format/path");
     if (e != cudaSuccess) return cuda_fail(e, "shared expert up kernel");

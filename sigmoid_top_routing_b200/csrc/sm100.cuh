@@ -35,10 +35,11 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false when the limit ran out (the caller records the error).
+// Bounded wait: false when `limit` polls ran out (the caller records the
+// error).  The pipelines pass kWaitLimit; a raised abort flag ends it early.
 constexpr uint32_t kWaitLimit = 1u << 24;
-MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
+MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag, uint32_t limit = kWaitLimit) {
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 1023u) == 1023u && abort_flag && *abort_flag) return false;
     }

@@ -23,6 +23,16 @@ Recipe (every workload):
     q = clip(round((w - bias) / scale), 0, 15); eight 4-bit codes per uint32,
     little-endian, the low nibble holding the lowest k.  The dequantised value
     is scale * q + bias.
+  * NVFP4 experts in the ModelOpt layout the pages name (TensorFold issue #548:
+    "weight uint8 [N, K/2], weight_scale e4m3 [N, K/16], weight_scale_2 as the
+    global scale"): per expert and projection a global scale
+    g = max|w| / (6 * 448) (fp32); per block of 16 along K a scale
+    s = max|w_block| / (6 * g) rounded to the nearest e4m3 code (ties to the
+    even code, at most 448); each weight w / (s * g) rounded to the nearest
+    e2m1 code (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; ties to the even code,
+    at most 6).  Two codes per byte, the low nibble holding the lower k.
+    Only the encoding lives here: it picks codes on the two grids below and
+    never turns a code back into a value.
 """
 from __future__ import annotations
 
@@ -33,7 +43,7 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "MoEInputs", "make_inputs", "f32_to_bf16_bits",
-    "bf16_bits_to_f32", "quantize_affine4_g64", "unpack_affine4",
+    "bf16_bits_to_f32", "quantize_affine4_g64", "unpack_affine4", "quantize_nvfp4",
 ]
 
 AFFINE_GROUP = 64
@@ -49,7 +59,7 @@ class Workload:
     k: int
     I: int
     act: str = "swiglu"          # "swiglu" | "relu2"
-    fmt: str = "bf16"            # "bf16" | "affine4"
+    fmt: str = "bf16"            # "bf16" | "affine4" | "nvfp4"
     eps: float = 1e-6
     router_scale: float = 1.0
     out_scale: float = 1.0
@@ -94,6 +104,9 @@ WORKLOADS = {
 for _T in (1, 8, 64, 512, 8192):
     WORKLOADS[f"affine4_t{_T}"] = Workload(f"affine4_t{_T}", T=_T, H=2048, E=64, k=4, I=1536,
                                            fmt="affine4")
+# the same block with NVFP4 experts (ModelOpt layout)
+for _T in (1, 8, 64, 512, 8192):
+    WORKLOADS[f"nvfp4_t{_T}"] = Workload(f"nvfp4_t{_T}", T=_T, H=2048, E=64, k=4, I=1536, fmt="nvfp4")
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -137,6 +150,60 @@ def quantize_affine4_g64(w: np.ndarray):
     return packed, scale_bits, bias_bits
 
 
+# Magnitudes of the e2m1 codes 0..7 (code = sign << 3 | magnitude index), and
+# of the finite non-negative e4m3 codes 0..126 (0x7F is NaN): the grids the
+# encoder rounds onto, ascending.
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+E4M3_GRID = np.array([m / 8.0 * 2.0 ** -6 for m in range(8)] +
+                     [(1.0 + m / 8.0) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)][:119])
+
+
+def _round_to_grid(a: np.ndarray, grid: np.ndarray) -> np.ndarray:
+    """Index of the nearest grid value to each |a| (ties to the even index),
+    saturating at the last entry.  Works in the precision of `a`: the grid's
+    midpoints are exact in float32."""
+    a = np.abs(np.asarray(a))
+    mid = ((grid[:-1] + grid[1:]) / 2).astype(a.dtype)
+    idx = np.searchsorted(mid, a, side="left")           # a == mid[j] gives j, the lower neighbour
+    tie = np.zeros(a.shape, dtype=bool)
+    inb = idx < len(mid)
+    tie[inb] = a[inb] == mid[idx[inb]]
+    return np.where(tie & (idx % 2 == 1), idx + 1, idx).astype(np.int64)
+
+
+def _round_e2m1(a: np.ndarray) -> np.ndarray:
+    """_round_to_grid(a, E2M1_GRID) in three rint regimes: on 2|a| the grid is
+    0..4 in steps of 1, then 4..8 in steps of 2, then 8..12 in steps of 4, and
+    np.rint rounds ties to even, which is the even code in each regime."""
+    a2 = 2 * np.abs(np.asarray(a, dtype=np.float32))
+    lo = np.rint(a2)
+    mid = np.rint(a2 / 2) + 2
+    hi = np.minimum(np.rint(a2 / 4), 3) + 4
+    return np.where(a2 < 4, lo, np.where(a2 < 8, mid, hi)).astype(np.int64)
+
+
+def quantize_nvfp4(w: np.ndarray):
+    """Encode an fp32 (N, K) weight as NVFP4 (ModelOpt layout).
+
+    Returns (codes uint8 (N, K/2), block scales uint8 e4m3 codes (N, K/16),
+    global scale float32).  Input encoding only."""
+    w = np.asarray(w, dtype=np.float32)
+    N, K = w.shape
+    assert K % 16 == 0
+    amax = float(np.abs(w).max())
+    g = np.float32(amax / (6.0 * 448.0)) if amax > 0 else np.float32(1.0)
+    blocks = w.reshape(N, K // 16, 16)
+    bmax = np.abs(blocks).max(axis=-1).astype(np.float64)
+    s_code = _round_to_grid(bmax / (6.0 * float(g)), E4M3_GRID)
+    s_val = E4M3_GRID[s_code]
+    denom = np.where(s_val == 0, 1.0, s_val * float(g)).astype(np.float32)[..., None]
+    mag = _round_e2m1(blocks / denom)
+    mag = np.where((s_val == 0)[..., None], 0, mag)
+    code = (mag | (np.signbit(blocks) & (mag != 0)).astype(np.int64) << 3).reshape(N, K)
+    packed = (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+    return packed, s_code.astype(np.uint8), g
+
+
 def unpack_affine4(packed: np.ndarray) -> np.ndarray:
     """Unpack (..., K/8) uint32 words into (..., K) 4-bit codes (uint8)."""
     p = np.asarray(packed, dtype=np.uint32)[..., None]
@@ -160,6 +227,8 @@ class MoEInputs:
     w2_q: Optional[np.ndarray] = None  # affine4: (E, H, I/8) uint32
     w2_scale: Optional[np.ndarray] = None
     w2_bias: Optional[np.ndarray] = None
+    w1_global: Optional[np.ndarray] = None   # nvfp4: (E,) fp32 global scale of W1 (weight_scale_2)
+    w2_global: Optional[np.ndarray] = None   # nvfp4: (E,) fp32 global scale of W2 (the down scale)
     nan_rows: Optional[np.ndarray] = None
     hot: Optional[np.ndarray] = None
     # shared expert (one expert, same format and activation, width shared_I):
@@ -180,18 +249,40 @@ def _normal_f32(rng: np.random.Generator, shape, std: float) -> np.ndarray:
 
 
 def _expert_weights(rng, E, N, K, fmt):
-    """Draw E experts' (N, K) weights one expert at a time (bounded memory)."""
+    """Draw E experts' (N, K) weights one expert at a time (in stream order)
+    and encode them; the encoding of different experts runs on a few threads
+    (numpy releases the GIL), which changes no value.
+    Returns (bf16 bits, codes, scales, biases or global scales)."""
     if fmt == "bf16":
         out = np.empty((E, N, K), dtype=np.uint16)
         for e in range(E):
             out[e] = f32_to_bf16_bits(_normal_f32(rng, (N, K), 0.02))
         return out, None, None, None
-    q = np.empty((E, N, K // 8), dtype=np.uint32)
-    s = np.empty((E, N, K // AFFINE_GROUP), dtype=np.uint16)
-    b = np.empty((E, N, K // AFFINE_GROUP), dtype=np.uint16)
-    for e in range(E):
-        q[e], s[e], b[e] = quantize_affine4_g64(_normal_f32(rng, (N, K), 0.02))
-    return None, q, s, b
+    import concurrent.futures as cf
+    import os
+    if fmt == "nvfp4":
+        q = np.empty((E, N, K // 2), dtype=np.uint8)
+        s = np.empty((E, N, K // 16), dtype=np.uint8)
+        g = np.empty(E, dtype=np.float32)
+    else:
+        q = np.empty((E, N, K // 8), dtype=np.uint32)
+        s = np.empty((E, N, K // AFFINE_GROUP), dtype=np.uint16)
+        g = np.empty((E, N, K // AFFINE_GROUP), dtype=np.uint16)
+    enc = quantize_nvfp4 if fmt == "nvfp4" else quantize_affine4_g64
+
+    def one(e, w):
+        q[e], s[e], g[e] = enc(w)
+
+    workers = max(1, min(8, os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        pending = []
+        for e in range(E):
+            pending.append(ex.submit(one, e, _normal_f32(rng, (N, K), 0.02)))
+            if len(pending) >= 2 * workers:      # bounded memory: at most 2x workers drafts alive
+                pending.pop(0).result()
+        for f in pending:
+            f.result()
+    return None, q, s, g
 
 
 def make_inputs(wl: Workload, *, with_experts: bool = True, hot_delta: Optional[float] = None) -> MoEInputs:
@@ -221,6 +312,9 @@ def make_inputs(wl: Workload, *, with_experts: bool = True, hot_delta: Optional[
     if with_experts:
         w1, q1, s1, b1 = _expert_weights(r_w1, E, n1, H, wl.fmt)
         w2, q2, s2, b2 = _expert_weights(r_w2, E, H, I, wl.fmt)
+    g1 = g2 = None
+    if wl.fmt == "nvfp4":                       # the fourth value is the global scale
+        g1, g2, b1, b2 = b1, b2, None, None
     shared = None
     if with_experts and wl.shared_I:
         Is = wl.shared_I
@@ -228,6 +322,9 @@ def make_inputs(wl: Workload, *, with_experts: bool = True, hot_delta: Optional[
         sw2, sq2, ss2, sb2 = _expert_weights(r_shared, 1, H, Is, wl.fmt)
         shared = {"w1_bits": sw1, "w2_bits": sw2, "w1_q": sq1, "w1_scale": ss1, "w1_bias": sb1,
                   "w2_q": sq2, "w2_scale": ss2, "w2_bias": sb2}
+        if wl.fmt == "nvfp4":                   # the fourth value is the global scale
+            shared.update(w1_global=sb1, w2_global=sb2, w1_bias=None, w2_bias=None)
     return MoEInputs(wl=wl, x_bits=f32_to_bf16_bits(x), w_router=w_router, expert_bias=bias,
                      w1_bits=w1, w2_bits=w2, w1_q=q1, w1_scale=s1, w1_bias=b1,
-                     w2_q=q2, w2_scale=s2, w2_bias=b2, nan_rows=nan_rows, hot=hot, shared=shared)
+                     w2_q=q2, w2_scale=s2, w2_bias=b2, w1_global=g1, w2_global=g2, nan_rows=nan_rows,
+                     hot=hot, shared=shared)

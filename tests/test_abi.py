@@ -155,7 +155,7 @@ def test_router_cfg_refuses_unknown_modes(lib):
         assert lib.moe_route_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, ctypes.byref(cfg),
                                 0x30000, 0x40000, None) == abi.MOE_ERR_UNSUPPORTED
         assert lib.moe_forward_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, 1.0,
-                                  ctypes.byref(cfg), None, ctypes.byref(_weights()), 0x30000, 0x40000,
+                                  ctypes.byref(cfg), None, None, ctypes.byref(_weights()), 0x30000, 0x40000,
                                   ctypes.byref(_plan()), 0x50000, 0x1000000, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
 
 
@@ -185,3 +185,42 @@ def test_dispatch_switch(lib):
     old = lib.moe_set_dispatch(abi.MOE_DISPATCH_GEMV)
     assert lib.moe_set_dispatch(99) == abi.MOE_DISPATCH_GEMV      # invalid value ignored
     assert lib.moe_set_dispatch(old) == abi.MOE_DISPATCH_GEMV
+
+
+def test_exec_cfg_is_per_call_and_validated(lib):
+    """The combine mode passed per call sizes the workspace whatever the
+    process-wide default is; values outside the enums are refused."""
+    d = _d()
+    atomic, ordered = abi.moe_exec_cfg(0, abi.MOE_COMBINE_ATOMIC), abi.moe_exec_cfg(0, abi.MOE_COMBINE_ORDERED)
+    n_a = lib.moe_workspace_bytes_ex(ctypes.byref(d), 0, ctypes.byref(atomic))
+    n_o = lib.moe_workspace_bytes_ex(ctypes.byref(d), 0, ctypes.byref(ordered))
+    assert n_o > n_a > 0
+    old = lib.moe_set_combine(abi.MOE_COMBINE_ORDERED)
+    try:
+        assert lib.moe_workspace_bytes_ex(ctypes.byref(d), 0, ctypes.byref(atomic)) == n_a
+        assert lib.moe_workspace_bytes_ex(ctypes.byref(d), 0, None) == n_o      # NULL: the process default
+    finally:
+        lib.moe_set_combine(old)
+    for bad in (abi.moe_exec_cfg(7, 0), abi.moe_exec_cfg(0, 5)):
+        assert lib.moe_workspace_bytes_ex(ctypes.byref(d), 0, ctypes.byref(bad)) == 0
+        assert lib.moe_experts_ex(0x10000, ctypes.byref(_plan()), 0x30000, ctypes.byref(d),
+                                  ctypes.byref(_weights()), ctypes.byref(bad), -1, None, 1.0, 0x20000,
+                                  0x1000000, n_o, None) == abi.MOE_ERR_UNSUPPORTED
+        assert lib.moe_forward_ex(0x10000, None, 0x20000, None, ctypes.byref(d), 1e-6, 1.0, 1.0, None,
+                                  ctypes.byref(bad), None, ctypes.byref(_weights()), 0x30000, 0x40000,
+                                  ctypes.byref(_plan()), 0x50000, 0x1000000, 1 << 30, None) == abi.MOE_ERR_UNSUPPORTED
+
+
+def test_experts_ex_refuses_bad_skip(lib):
+    d = _d()
+    n = lib.moe_workspace_bytes(ctypes.byref(d), 0)
+
+    def call(skip, dd=d):
+        return lib.moe_experts_ex(0x10000, ctypes.byref(_plan()), 0x30000, ctypes.byref(dd),
+                                  ctypes.byref(_weights()), None, skip, None, 1.0, 0x20000, 0x1000000, n, None)
+    assert call(-2) == abi.MOE_ERR_SHAPE
+    assert call(d.E) == abi.MOE_ERR_SHAPE
+    assert "skip_expert" in lib.moe_last_error().decode()
+    assert call(0, _d(E=1, k=1)) == abi.MOE_ERR_SHAPE
+    assert lib.moe_experts_ex(0x10000, ctypes.byref(_plan()), 0x30000, ctypes.byref(d), ctypes.byref(_weights()),
+                              None, -1, 0x40004, 1.0, 0x20000, 0x1000000, n, None) == abi.MOE_ERR_ALIGN

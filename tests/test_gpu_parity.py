@@ -125,6 +125,22 @@ def test_nan_logit_rows_via_logits_argument(api):
     assert rep.nan_rows == 2
 
 
+def test_nan_logit_rows_via_logits_argument_tcgen05_prefill(api):
+    """The prefill workload at full size with 1 % of router-logit rows all-NaN
+    passed through the logits argument, on the library's own choice of expert
+    kernels (the tcgen05 grouped GEMM at this size)."""
+    import oracle as O
+    wl = dataclasses.replace(G.WORKLOADS["lfm2_prefill_t4096"], nan_rows=0)
+    inp = inputs_of(wl)
+    L = O.router_logits(inp.x_bits, inp.w_router).astype(np.float32)
+    rows = np.sort(np.random.default_rng(5).choice(wl.T, 41, replace=False))
+    L[rows] = np.nan
+    out = run_forward(api, inp, logits=L)
+    assert np.all(out["idx"][rows] == np.arange(wl.k))
+    rep = _check_all(inp, out, logits=L)
+    assert rep.nan_rows == 41
+
+
 def test_nan_token_rows_prefill_shape(api):
     from sigmoid_top_routing_b200 import abi
     inp = inputs_of(_small("lfm2_prefill_t4096", 300))
