@@ -10,8 +10,8 @@ the C ABI with the workspace filled with 0xFF before the launches:
     for bit; atomic combine: the same up to the order of fp32 additions);
   * the plan is the oracle's plan over E + 1 experts, bit for bit;
   * y matches the oracle's skip form (experts_block) on the GPU's picks.
-A skip in the middle of the expert range (weights for every plan expert,
-one of them left out) is checked against the oracle too."""
+A skip of the most-routed expert, with weights for every plan expert, is
+checked against the oracle too."""
 import numpy as np
 import pytest
 
@@ -143,7 +143,6 @@ def test_skip_below_the_last_expert(api, name, T, dispatch):
     idx, w = api.moe_route(D.x, None, D.w_router, D.expert_bias, E=wl.E, k=wl.k, eps=wl.eps, scale=wl.router_scale)
     idx_np = idx.cpu().numpy().astype(np.int64)
     skip = int(np.bincount(idx_np.ravel(), minlength=wl.E).argmax())
-    assert 0 < skip < wl.E - 1 or wl.E - 1 > skip >= 0
     plan = api.moe_plan(idx, E=wl.E, H=wl.H, I=wl.I)
     y = api.moe_experts(D.x, plan, w, D.W, E=wl.E, I=wl.I, out_scale=wl.out_scale, skip=skip, dispatch=disp)
     torch.cuda.synchronize()
