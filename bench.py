@@ -45,7 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "bf16_tflops": 2250.0}
 DEFAULT_WORKLOAD = "lfm2_prefill_t4096"
 SIDE_WORKLOADS = ("lfm2_decode_t8", "nemotron_relu2_t2048", "affine4_t1", "affine4_t8", "affine4_t64",
-                  "affine4_t512", "affine4_t8192")
+                  "affine4_t512", "affine4_t8192", "nvfp4_t1", "nvfp4_t8", "nvfp4_t64", "nvfp4_t512",
+                  "nvfp4_t8192")
 GRAPH_BLOCK = 32      # steps per captured graph (at most; fewer when K is smaller)
 
 
@@ -106,10 +107,13 @@ def config_of(wl, args) -> dict:
 # ----------------------------------------------------------------------------- algorithmic work
 
 def expert_bytes(wl) -> tuple:
-    """(W1 bytes, W2 bytes) of one expert: bf16, or 4-bit codes + bf16 scale and bias per 64."""
+    """(W1 bytes, W2 bytes) of one expert: bf16; affine 4-bit codes + bf16 scale and
+    bias per 64; NVFP4 codes + an e4m3 scale per 16 + an fp32 global scale."""
     n1 = (2 if wl.act == "swiglu" else 1) * wl.I
     if wl.fmt == "bf16":
         return n1 * wl.H * 2, wl.H * wl.I * 2
+    if wl.fmt == "nvfp4":
+        return n1 * wl.H // 2 + n1 * wl.H // 16 + 4, wl.H * wl.I // 2 + wl.H * wl.I // 16 + 4
     return n1 * wl.H // 2 + (n1 * wl.H // 64) * 4, wl.H * wl.I // 2 + (wl.H * wl.I // 64) * 4
 
 
@@ -391,7 +395,8 @@ class Inputs:
             return self.host[k]
         src = self.host[k]
         inp = self.G.make_inputs(wl, with_experts=False)
-        for f in ("w1_bits", "w2_bits", "w1_q", "w1_scale", "w1_bias", "w2_q", "w2_scale", "w2_bias", "shared"):
+        for f in ("w1_bits", "w2_bits", "w1_q", "w1_scale", "w1_bias", "w2_q", "w2_scale", "w2_bias", "w1_global",
+                  "w2_global", "shared"):
             setattr(inp, f, getattr(src, f))
         return inp
 
@@ -404,15 +409,7 @@ class Inputs:
             w1, w2 = expert_bytes(inp.wl)
             all_w = (w1 + w2) * inp.wl.E
             n_sets = max(2, min(16, math.ceil(4 * L2_BYTES / all_w)))
-            sets = [W]
-            for _ in range(n_sets - 1):
-                sets.append(self.api.ExpertWeights(
-                    act=W.act, fmt=W.fmt, w1=W.w1.clone(), w2=W.w2.clone(),
-                    w1_scale=None if W.w1_scale is None else W.w1_scale.clone(),
-                    w1_bias=None if W.w1_bias is None else W.w1_bias.clone(),
-                    w2_scale=None if W.w2_scale is None else W.w2_scale.clone(),
-                    w2_bias=None if W.w2_bias is None else W.w2_bias.clone(),
-                    swiglu_limit=W.swiglu_limit))
+            sets = [W] + [W.clone() for _ in range(n_sets - 1)]
             self.dev[k] = (sets, all_w)
         return self.dev[k]
 
@@ -557,6 +554,12 @@ class Runner:
         return out
 
 
+def dtype_of(wl) -> str:
+    """The arithmetic the path computes in: bf16 operands, or 4-bit weight codes
+    dequantised on chip against bf16 activations; fp32 accumulation throughout."""
+    return {"bf16": "bf16", "affine4": "u4+bf16", "nvfp4": "e2m1+bf16"}[wl.fmt]
+
+
 def gemv_path_of(wl, dispatch: str) -> bool:
     """The library's AUTO choice: affine 4-bit experts at <= 8 pairs per expert take the GEMV."""
     return dispatch == "gemv" or (dispatch == "auto" and wl.fmt != "bf16" and wl.T * wl.k <= 8 * wl.E
@@ -646,7 +649,7 @@ def main():
     value = job_rate(wl.T * K, world, ms / 1e3)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if wl.fmt == "bf16" else "u4+bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": dtype_of(wl), "data": "synthetic",
             "config": config_of(wl, args),
             "l2_detail": f"{R.n_sets} weight copies rotated ({R.n_sets * R.all_w / 1e9:.2f} GB), "
                          f"{R.wm['active_experts']} active experts per step",
@@ -699,7 +702,7 @@ def main():
         up2 = float(max_over_ranks(r.stage_ms(k2) * 1e3, dist, world, "cuda", torch.float64))
         c2 = sampler.summary(ta, tb)
         entry = {"value": job_rate(w2.T * k2, world, ms2 / 1e3), "unit": "tokens/s", "steps": k2,
-                 "ms_per_step": ms2 / k2, "dtype": "bf16" if w2.fmt == "bf16" else "u4+bf16",
+                 "ms_per_step": ms2 / k2, "dtype": dtype_of(w2),
                  "config": config_of(w2, args), "gpu_launches": r.launches * k2,
                  "roofline": roofline_of(r.wm, up2, pk, pk_kind, traffic_of("up", name)),
                  "step_roofline": step_roofline_of(r.wm, 1e3 * ms2 / k2, pk),

@@ -78,7 +78,7 @@ typedef enum {
 } moe_status;
 
 typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU2 = 1 } moe_act;
-typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1 } moe_wfmt;
+typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1, MOE_W_NVFP4 = 2 } moe_wfmt;
 
 /* Which expert kernels run (per call through moe_exec_cfg, or the process-wide
  * default of moe_set_dispatch). */
@@ -111,6 +111,18 @@ typedef struct {
  *     w2 = codes (E, H, I/8) uint32, w2_scale, w2_bias = (E, H, I/64) bf16.
  *     A uint32 holds 8 consecutive k, the low nibble first; the weight is
  *     scale * q + bias (TensorFold pull #1492, "What": Affine4 experts).
+ *   fmt = MOE_W_NVFP4 (ModelOpt NVFP4, read as stored, W4A16: TensorFold
+ *     issue #548, "weight uint8 [N, K/2], weight_scale e4m3 [N, K/16],
+ *     weight_scale_2 as the global scale", and the down projection's own
+ *     global scale):
+ *     w1 = codes (E, N1, H/2) uint8, two e2m1 codes per byte, the low nibble
+ *     the lower k; w1_scale = (E, N1, H/16) e4m3 bytes; w1_global = (E) fp32;
+ *     w2 = codes (E, H, I/2), w2_scale = (E, H, I/16), w2_global = (E) fp32;
+ *     the weight is e2m1(q) * e4m3(scale) * global.  *_bias are unused.
+ *     Kernels dequantise e2m1 * e4m3 exactly (into bf16 for the tcgen05
+ *     GEMM, into f16 for the decode GEMV, whose token rows are staged in f16
+ *     after an exact per-token power-of-two scale) and apply the global scale
+ *     to the fp32 sum.
  *   swiglu_limit (SWIGLU only; 0 = off, must be >= 0 and finite): before the
  *     activation the gate is clamped from above, g = min(g, limit), and the
  *     up value on both sides, u = clamp(u, -limit, limit); NaN stays NaN
@@ -126,6 +138,8 @@ typedef struct {
     const void* w2_scale;
     const void* w2_bias;
     float swiglu_limit;
+    const float* w1_global; /* MOE_W_NVFP4 only (else unused, may be NULL) */
+    const float* w2_global;
 } moe_experts_w;
 
 /* Router variants (TensorFold issue #548: the pieces each model family

@@ -18,7 +18,7 @@ MOE_OK, MOE_ERR_NULL, MOE_ERR_SHAPE, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED, MOE_ERR
 STATUS_NAMES = ["MOE_OK", "MOE_ERR_NULL", "MOE_ERR_SHAPE", "MOE_ERR_ALIGN", "MOE_ERR_UNSUPPORTED",
                 "MOE_ERR_WORKSPACE", "MOE_ERR_CUDA", "MOE_ERR_DEVICE"]
 MOE_ACT_SWIGLU, MOE_ACT_RELU2 = 0, 1
-MOE_W_BF16, MOE_W_AFFINE4_G64 = 0, 1
+MOE_W_BF16, MOE_W_AFFINE4_G64, MOE_W_NVFP4 = 0, 1, 2
 MOE_DISPATCH_AUTO, MOE_DISPATCH_GEMV, MOE_DISPATCH_GEMM = 0, 1, 2
 MOE_COMBINE_ATOMIC, MOE_COMBINE_ORDERED = 0, 1
 MOE_SCORE_SIGMOID, MOE_SCORE_SOFTMAX = 0, 1
@@ -34,7 +34,7 @@ class moe_experts_w(ctypes.Structure):
     _fields_ = [("fmt", c_int32), ("act", c_int32),
                 ("w1", c_void_p), ("w1_scale", c_void_p), ("w1_bias", c_void_p),
                 ("w2", c_void_p), ("w2_scale", c_void_p), ("w2_bias", c_void_p),
-                ("swiglu_limit", c_float)]
+                ("swiglu_limit", c_float), ("w1_global", c_void_p), ("w2_global", c_void_p)]
 
 
 class moe_router_cfg(ctypes.Structure):

@@ -48,7 +48,7 @@ def _stream(stream) -> int:
 class ExpertWeights:
     """Device tensors of the experts (layouts as in include/moe.h)."""
     act: int                          # abi.MOE_ACT_SWIGLU | abi.MOE_ACT_RELU2
-    fmt: int                          # abi.MOE_W_BF16 | abi.MOE_W_AFFINE4_G64
+    fmt: int                          # abi.MOE_W_BF16 | abi.MOE_W_AFFINE4_G64 | abi.MOE_W_NVFP4
     w1: torch.Tensor
     w2: torch.Tensor
     w1_scale: Optional[torch.Tensor] = None
@@ -56,10 +56,20 @@ class ExpertWeights:
     w2_scale: Optional[torch.Tensor] = None
     w2_bias: Optional[torch.Tensor] = None
     swiglu_limit: float = 0.0
+    w1_global: Optional[torch.Tensor] = None   # NVFP4: (E,) fp32 global scales
+    w2_global: Optional[torch.Tensor] = None
 
     def c_struct(self) -> abi.moe_experts_w:
         return abi.moe_experts_w(self.fmt, self.act, _ptr(self.w1), _ptr(self.w1_scale), _ptr(self.w1_bias),
-                                 _ptr(self.w2), _ptr(self.w2_scale), _ptr(self.w2_bias), self.swiglu_limit)
+                                 _ptr(self.w2), _ptr(self.w2_scale), _ptr(self.w2_bias), self.swiglu_limit,
+                                 _ptr(self.w1_global), _ptr(self.w2_global))
+
+    def clone(self) -> "ExpertWeights":
+        c = lambda t: None if t is None else t.clone()  # noqa: E731
+        return ExpertWeights(act=self.act, fmt=self.fmt, w1=c(self.w1), w2=c(self.w2), w1_scale=c(self.w1_scale),
+                             w1_bias=c(self.w1_bias), w2_scale=c(self.w2_scale), w2_bias=c(self.w2_bias),
+                             swiglu_limit=self.swiglu_limit, w1_global=c(self.w1_global),
+                             w2_global=c(self.w2_global))
 
 
 def router_cfg(score: str = "sigmoid", norm_topk: bool = True) -> abi.moe_router_cfg:

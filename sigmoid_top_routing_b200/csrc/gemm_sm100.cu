@@ -41,6 +41,7 @@
 #include "internal.h"
 #include "launch.h"
 #include "plan_dev.cuh"
+#include "quant.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -69,8 +70,9 @@ struct GemmParams {
     int K;                   // reduction length: H (up) or I (down)
     int rows_per_expert;     // rows of the A tensor per expert: 2I, I or H
     int feats;               // output features per expert: I (up) or H (down)
-    const uint16_t* wscale;  // affine 4-bit: (E, rows_per_expert, K/64) bf16 scales
-    const uint16_t* wbias;   //                and biases
+    const uint16_t* wscale;  // affine 4-bit: (E, rows_per_expert, K/64) bf16 scales; NVFP4: (.., K/16) e4m3 bytes
+    const uint16_t* wbias;   // affine 4-bit biases
+    const float* wglobal;    // NVFP4: (E) fp32 global scale, multiplied into the fp32 sum
     float swiglu_limit;      // up SwiGLU: clamp of the gate (above) and up (both sides); 0 off
     int skip;                // plan expert given no tiles (its pairs are computed nowhere), or -1
     int E_w;                 // experts the weight tensor holds
@@ -175,6 +177,29 @@ MOE_DEV void dequant_chunks(const uint32_t* codes, int c0, uint16_t scale, uint1
             const __nv_bfloat162 v = __hfma2(q2, s2, b2);
             o[p] = *reinterpret_cast<const uint32_t*>(&v);
         }
+        *reinterpret_cast<uint4*>(arow + (((c ^ (r & 7)) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// NVFP4: chunks [c0, c0 + NC) of one 128-byte A row from 8 e2m1 codes each
+// (one 32-bit word, the low nibble first) and the row's four e4m3 block scales
+// of this k-block (byte b serves chunks 2b and 2b + 1).  The code pairs and the
+// scale convert exactly to f16, their f16 product is exact (at most six
+// significant bits, in range), and widening to fp32 then rounding the pair to
+// bf16 is exact again: A holds e2m1 * e4m3 exactly; the global scale is applied
+// to the fp32 sum in the epilogue.
+template <int NC>
+MOE_DEV void dequant_nvfp4_chunks(const uint32_t* codes, int c0, uint32_t scales4, unsigned char* arow, int r) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+        const int c = c0 + i;
+        const uint32_t sb = (scales4 >> (8 * (c >> 1))) & 0xFFu;
+        const uint32_t s2 = e4m3x2_to_f16x2(sb | (sb << 8));
+        uint32_t p[4];
+        e2m1x8_to_f16(codes[i], p);
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[j] = f16x2_to_bf16x2(hmul2_u32(p[j], s2));
         *reinterpret_cast<uint4*>(arow + (((c ^ (r & 7)) & 7) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
@@ -465,9 +490,15 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         auto issue = [&](int slot) {
             if (at < total) {
                 const size_t gr = grow(atl);
-                const size_t gi = gr < nrows ? gr * G + akb : 0;
-                cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt), g.wscale + (gi & ~size_t(1)));
-                cp_async4(smem_u32(s_sb + (slot * 2 + 1) * 256 + dt), g.wbias + (gi & ~size_t(1)));
+                if (WFMT == 2) {      // the row's four e4m3 block scales of this k-block: one word
+                    const size_t wi = gr < nrows ? gr * (size_t)(g.K / 16) + 4 * (size_t)akb : 0;
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt),
+                              reinterpret_cast<const uint8_t*>(g.wscale) + wi);
+                } else {
+                    const size_t gi = gr < nrows ? gr * G + akb : 0;
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt), g.wscale + (gi & ~size_t(1)));
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 1) * 256 + dt), g.wbias + (gi & ~size_t(1)));
+                }
                 if (++akb == atl.kb1) {
                     at += gridDim.x;
                     if (at < total) {
@@ -507,7 +538,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     cw[4 * q + 2] = c4.z;
                     cw[4 * q + 3] = c4.w;
                 }
-                dequant_chunks<kCPT>(cw, cbeg, sc, bi, sA + size_t(s) * kAStage + r * 128, r);
+                if (WFMT == 2)
+                    dequant_nvfp4_chunks<kCPT>(cw, cbeg, inb ? sw : 0u, sA + size_t(s) * kAStage + r * 128, r);
+                else
+                    dequant_chunks<kCPT>(cw, cbeg, sc, bi, sA + size_t(s) * kAStage + r * 128, r);
                 fence_proxy_async_smem();                 // generic-proxy writes -> tensor core reads
                 mbar_arrive(&full[s]);
                 if (++s == STAGES) { s = 0; ph ^= 1; }
@@ -550,6 +584,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tbase = tmem_base + (uint32_t(32 * sub) << 16) + buf * (kDual ? 2 * BN : BN);
+            const float gsc = WFMT == 2 ? __ldg(g.wglobal + tl.e) : 1.0f;
             for (int c0 = 0; c0 < tl.n; c0 += 16) {
                 float v[16];
                 if (dead) {
@@ -557,6 +592,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     for (int i = 0; i < 16; ++i) v[i] = 0.0f;
                 } else {
                     tmem_ld16(tbase + c0, v);
+                    if (WFMT == 2) {      // NVFP4: the expert's global scale on the fp32 sum
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] *= gsc;
+                    }
                 }
                 if (MODE == kDown) {
                     const int f = tl.wt * 128 + lrow;
@@ -591,6 +630,10 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                         for (int i = 0; i < 16; ++i) u[i] = 0.0f;
                     } else {
                         tmem_ld16(tbase + BN + c0, u);
+                        if (WFMT == 2) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) u[i] *= gsc;
+                        }
                     }
                     const int f = tl.wt * 128 + lrow;
                     if (!dead && f < g.feats) {
@@ -745,6 +788,7 @@ GemmParams params(const ExpertArgs& a, bool up) {
         g.feats = a.I;
         g.wscale = a.w1_scale;
         g.wbias = a.w1_bias;
+        g.wglobal = a.w1_global;
         g.swiglu_limit = a.swiglu_limit;
     } else {
         g.K = a.I;
@@ -752,6 +796,7 @@ GemmParams params(const ExpertArgs& a, bool up) {
         g.feats = a.H;
         g.wscale = a.w2_scale;
         g.wbias = a.w2_bias;
+        g.wglobal = a.w2_global;
     }
     return g;
 }
@@ -780,6 +825,29 @@ cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     return launch_k(k_gather_rows, dim3(blocks), dim3(256), 0, s, pdl, a.x, a.perm, a.xs, P, a.k, a.H);
 }
 
+namespace {
+
+// 4-bit experts (WFMT 1 affine, 2 NVFP4): codes dequantised on chip.
+template <int WFMT>
+cudaError_t gemm_up_q4(const ExpertArgs& a, const GemmParams& g, int bn, bool pdl, cudaStream_t s) {
+    if (a.act == 0) {
+        if (bn == 32) return run<kUpSwiglu, 32, 8, WFMT>(a, g, a.w1, pdl, s);
+        return run<kUpSwiglu, 128, 3, WFMT>(a, g, a.w1, pdl, s);
+    }
+    if (bn == 32) return run<kUpRelu2, 32, 8, WFMT>(a, g, a.w1, pdl, s);
+    if (bn == 128) return run<kUpRelu2, 128, 5, WFMT>(a, g, a.w1, pdl, s);
+    return run<kUpRelu2, 256, 4, WFMT>(a, g, a.w1, pdl, s);
+}
+
+template <int WFMT>
+cudaError_t gemm_down_q4(const ExpertArgs& a, const GemmParams& g, int bn, bool pdl, cudaStream_t s) {
+    if (bn == 32) return run<kDown, 32, 8, WFMT>(a, g, a.w2, pdl, s);
+    if (bn == 128) return run<kDown, 128, 5, WFMT>(a, g, a.w2, pdl, s);
+    return run<kDown, 256, 4, WFMT>(a, g, a.w2, pdl, s);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const GemmParams g = params(a, true);
     const int bn = pick_bn(a);
@@ -792,13 +860,9 @@ cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
         if (bn == 128) return run<kUpRelu2, 128, 5, 0>(a, g, a.w1, pdl, s);
         return run<kUpRelu2, 256, 4, 0>(a, g, a.w1, pdl, s);
     }
-    if (a.act == 0) {
-        if (bn == 32) return run<kUpSwiglu, 32, 8, 1>(a, g, a.w1, pdl, s);
-        return run<kUpSwiglu, 128, 3, 1>(a, g, a.w1, pdl, s);
-    }
-    if (bn == 32) return run<kUpRelu2, 32, 8, 1>(a, g, a.w1, pdl, s);
-    if (bn == 128) return run<kUpRelu2, 128, 5, 1>(a, g, a.w1, pdl, s);
-    return run<kUpRelu2, 256, 4, 1>(a, g, a.w1, pdl, s);
+    if (a.fmt == 1) return gemm_up_q4<1>(a, g, bn, pdl, s);
+    if (a.fmt == 2) return gemm_up_q4<2>(a, g, bn, pdl, s);
+    return cudaErrorNotSupported;
 }
 
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
@@ -809,9 +873,9 @@ cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
         if (bn == 128) return run<kDown, 128, 5, 0>(a, g, a.w2, pdl, s);
         return run<kDown, 256, 4, 0>(a, g, a.w2, pdl, s);
     }
-    if (bn == 32) return run<kDown, 32, 8, 1>(a, g, a.w2, pdl, s);
-    if (bn == 128) return run<kDown, 128, 5, 1>(a, g, a.w2, pdl, s);
-    return run<kDown, 256, 4, 1>(a, g, a.w2, pdl, s);
+    if (a.fmt == 1) return gemm_down_q4<1>(a, g, bn, pdl, s);
+    if (a.fmt == 2) return gemm_down_q4<2>(a, g, bn, pdl, s);
+    return cudaErrorNotSupported;
 }
 
 }  // namespace moe

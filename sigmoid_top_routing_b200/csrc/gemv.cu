@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(256) k_zero(float* p, size_t n4) {
 
 // Persistent grids: two CTAs of 8 warps per SM.
 cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    if (a.fmt == 1) return launch_gemv_affine_up(a, pdl, s);
+    if (a.fmt == 1 || a.fmt == 2) return launch_gemv_q4_up(a, pdl, s);
     if (a.fmt != 0) return cudaErrorNotSupported;
     const int grid = device_info().sm_count * 2;
     if (a.act == 0) return launch_k(k_gemv_up<0>, dim3(grid), dim3(kWarps * 32), 0, s, pdl, a);
@@ -284,7 +284,7 @@ cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
 }
 
 cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    if (a.fmt == 1) return launch_gemv_affine_down(a, pdl, s);
+    if (a.fmt == 1 || a.fmt == 2) return launch_gemv_q4_down(a, pdl, s);
     if (a.fmt != 0) return cudaErrorNotSupported;
     const int grid = device_info().sm_count * 2;
     return launch_k(k_gemv_down, dim3(grid), dim3(kWarps * 32), 0, s, pdl, a);

@@ -51,7 +51,7 @@ struct ExpertArgs {
     int E_w;                 // experts the weight tensors hold (E, or E - 1 when the last is skipped)
     int skip;                // plan expert whose pairs are computed nowhere and left out, or -1
     int act;                 // 0 swiglu, 1 relu2
-    int fmt;                 // 0 bf16, 1 affine4
+    int fmt;                 // 0 bf16, 1 affine4, 2 nvfp4
     float swiglu_limit;      // > 0: g = min(g, L), u = clamp(u, -L, L) before silu(g) * u
     const void* w1;
     const uint16_t* w1_scale;
@@ -59,6 +59,8 @@ struct ExpertArgs {
     const void* w2;
     const uint16_t* w2_scale;
     const uint16_t* w2_bias;
+    const float* w1_global;  // NVFP4: (E) fp32 global scales of W1 and W2
+    const float* w2_global;
     uint16_t* h;             // (P, I) bf16 in plan order
     uint16_t* xs;            // (P, H) bf16 gathered rows (GEMM path)
     float* y_acc;            // (T, H) fp32, or (P, H) weighted slot outputs when ordered
@@ -85,13 +87,15 @@ cudaError_t launch_plan(const PlanArgs& a, bool pdl, cudaStream_t s, int* n_laun
 size_t plan_scratch_ints(int P, int E);
 cudaError_t launch_gemv_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
-// Affine 4-bit GEMV (codes dequantised in registers); launch_gemv_up/down
-// route fmt == 1 here.
-cudaError_t launch_gemv_affine_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
-cudaError_t launch_gemv_affine_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
-// MOE_DISPATCH_AUTO's choice: the GEMV for affine 4-bit experts with at most
-// this many routed pairs per expert on average, the tcgen05 GEMM otherwise.
+// 4-bit GEMV (affine or NVFP4 codes dequantised in registers, K <= 8192);
+// launch_gemv_up/down route fmt 1 and 2 here.
+cudaError_t launch_gemv_q4_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemv_q4_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// MOE_DISPATCH_AUTO's choice: the GEMV for 4-bit experts with at most this
+// many routed pairs per expert on average, the tcgen05 GEMM otherwise.
 constexpr int kAffineGemvMaxPairsPerExpert = 8;
+// Whether the tcgen05 GEMM runs NVFP4 experts in this build.
+constexpr bool kNvfp4Gemm = true;
 // The tcgen05 grouped GEMMs (cudaErrorNotSupported where a format has none).
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);

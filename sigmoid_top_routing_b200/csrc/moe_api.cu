@@ -81,7 +81,7 @@ moe_status check_dims(const moe_dims* d) {
 }
 
 moe_status check_fmt(int32_t fmt) {
-    if (fmt != MOE_W_BF16 && fmt != MOE_W_AFFINE4_G64)
+    if (fmt != MOE_W_BF16 && fmt != MOE_W_AFFINE4_G64 && fmt != MOE_W_NVFP4)
         return fail(MOE_ERR_UNSUPPORTED, "weight format %d", fmt);
     return MOE_OK;
 }
@@ -178,6 +178,14 @@ moe_status check_weights(const moe_experts_w* W) {
             !aligned16(W->w2_bias))
             return fail(MOE_ERR_ALIGN, "affine-4 scale/bias not 16-byte aligned");
     }
+    if (W->fmt == MOE_W_NVFP4) {
+        if (!W->w1_scale || !W->w2_scale || !W->w1_global || !W->w2_global)
+            return fail(MOE_ERR_NULL, "NVFP4 block-scale or global-scale pointer is NULL");
+        if (!aligned16(W->w1_scale) || !aligned16(W->w2_scale))
+            return fail(MOE_ERR_ALIGN, "NVFP4 block scales not 16-byte aligned");
+        if ((reinterpret_cast<uintptr_t>(W->w1_global) | reinterpret_cast<uintptr_t>(W->w2_global)) & 3u)
+            return fail(MOE_ERR_ALIGN, "NVFP4 global scales not 4-byte aligned");
+    }
     if (!(W->swiglu_limit >= 0.0f) || W->swiglu_limit > 3.0e38f)
         return fail(MOE_ERR_SHAPE, "swiglu_limit must be finite and >= 0 (0 = off)");
     return MOE_OK;
@@ -212,7 +220,8 @@ moe_status check_route_args(const void* x, const float* logits, const float* w_r
 // the codes faster than the GEMM's shared-memory dequant pipeline.
 bool use_gemv(const moe_dims* d, int32_t fmt, int mode) {
     if (mode != MOE_DISPATCH_AUTO) return mode == MOE_DISPATCH_GEMV;
-    return fmt == MOE_W_AFFINE4_G64 && d->H <= 8192 && d->I <= 8192 &&
+    if (fmt == MOE_W_NVFP4 && !kNvfp4Gemm) return true;   // no tcgen05 NVFP4 path in this build
+    return (fmt == MOE_W_AFFINE4_G64 || fmt == MOE_W_NVFP4) && d->H <= 8192 && d->I <= 8192 &&
            (size_t)d->T * d->k <= (size_t)kAffineGemvMaxPairsPerExpert * d->E;
 }
 
@@ -243,6 +252,8 @@ ExpertArgs make_expert_args(const void* x, const moe_plan_t* plan, const float* 
     a.w2 = W->w2;
     a.w2_scale = static_cast<const uint16_t*>(W->w2_scale);
     a.w2_bias = static_cast<const uint16_t*>(W->w2_bias);
+    a.w1_global = W->fmt == MOE_W_NVFP4 ? W->w1_global : nullptr;
+    a.w2_global = W->fmt == MOE_W_NVFP4 ? W->w2_global : nullptr;
     a.h = v.h;
     a.xs = v.xs;
     a.y_acc = v.y_acc;

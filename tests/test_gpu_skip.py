@@ -65,7 +65,7 @@ def _oracle_gate(inp, idx, w, y_bits, skip):
 
 CASES = [("lfm2_decode_t8", None, "gemm"), ("lfm2_decode_t8", None, "gemv"),
          ("lfm2_prefill_t4096", 300, "auto"), ("nemotron_relu2_t2048", 200, "auto"),
-         ("affine4_t64", None, "auto"), ("affine4_t512", None, "gemm")]
+         ("affine4_t64", None, "auto"), ("affine4_t512", None, "gemm"), ("nvfp4_t64", None, "auto")]
 
 
 @pytest.mark.parametrize("combine", ["ordered", "atomic"])
