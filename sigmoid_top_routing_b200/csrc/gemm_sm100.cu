@@ -52,7 +52,8 @@ using namespace sm100;
 constexpr int kBK = 64;                  // k per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kARows = 128 * kBK * 2;    // 16 KB: 128 weight rows of one k-block
 constexpr int kThreads = 192;            // bf16 weights: producer, MMA, 4 epilogue warps
-constexpr int kThreadsA4 = 448;          // affine 4-bit weights: + 8 dequantisation warps
+constexpr int kDq = 256;                 // 4-bit weights: dequantisation threads (8 warps)
+constexpr int kThreadsA4 = 192 + kDq;    // 4-bit weights: producer, MMA, 4 epilogue warps + dequant warps
 constexpr int kSBDepth = 4;              // stages of scales/biases in flight per dequant thread
 
 enum Mode { kUpSwiglu = 0, kUpRelu2 = 1, kDown = 2 };
@@ -81,9 +82,9 @@ struct GemmParams {
 };
 
 template <int BN, int STAGES, int ASTAGE, int CSTAGE, bool USE_U,
-          int SBRING = (CSTAGE ? kSBDepth * 2 * 256 * 4 : 0)>
+          int SBRING = (CSTAGE ? kSBDepth * 2 * kDq * 4 : 0), int BROWS = BN>
 struct Smem {
-    static constexpr int kBStage = BN * 128;
+    static constexpr int kBStage = BROWS * 128;                              // token rows of one stage
     static constexpr size_t kA = 0;
     static constexpr size_t kB = kA + size_t(STAGES) * ASTAGE;
     static constexpr size_t kC = kB + size_t(STAGES) * kBStage;             // packed 4-bit codes (affine)
@@ -98,6 +99,30 @@ struct Smem {
     static constexpr size_t kSB = kCnt + 513 * 4 + 12;                        // scale/bias ring (affine)
     static constexpr size_t kEnd = kSB + SBRING;
     static constexpr size_t kBytes = kEnd + 1024;                             // + alignment slack
+};
+
+// How a tile's A rows are laid out; the kernel and its host launcher both
+// derive the shared-memory layout from here.
+//   dual   SwiGLU, bf16, token tiles >= 64: 128 gate + 128 up rows, two accumulators
+//   inter  SwiGLU, 4-bit, token tiles >= 64: 64 features; in each 32-row TMEM
+//          quarter rows 0-15 are gate rows and 16-31 the matching up rows, so gate
+//          and up of a feature meet by one warp shuffle; one accumulator, so token
+//          tiles reach 256 and each dequantised A stage serves twice the tokens
+//   halves SwiGLU, token tiles of 32: 64 gate rows then 64 up rows, one accumulator,
+//          the halves meet through shared memory
+//   pair   (PAIR = 1) two CTAs on neighbouring SMs run one M = 256 MMA
+//          (tcgen05 cta_group::2): each holds its own 128 weight rows and half of
+//          the tile's token rows, and gets its 128 rows of the accumulator
+template <int MODE, int BN, int WFMT, int PAIR = 0>
+struct Cfg {
+    static constexpr int kBRows = PAIR ? BN / 2 : BN;       // token rows a CTA stages per k-block
+    static constexpr bool kInter = MODE == kUpSwiglu && WFMT != 0 && BN >= 64;
+    static constexpr bool kDual = MODE == kUpSwiglu && BN >= 64 && !kInter;
+    static constexpr bool kHalves = MODE == kUpSwiglu && BN < 64;
+    static constexpr int kAStage = kDual ? 2 * kARows : kARows;
+    static constexpr int kCStage = WFMT ? kAStage / 4 : 0;   // packed 4-bit codes of one A stage
+    static constexpr int kFpt = MODE == kUpSwiglu && !kDual ? 64 : 128;   // output features per tile
+    static constexpr uint32_t kABox = MODE == kUpSwiglu && !kDual ? 64 : 128;   // A rows per TMA box
 };
 
 struct Tile {
@@ -211,20 +236,23 @@ MOE_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memo
 template <int N>
 MOE_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int MODE, int BN, int STAGES, int WFMT>
+template <int MODE, int BN, int STAGES, int WFMT, int PAIR>
 __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams g) {
     // SwiGLU with wide token tiles keeps two accumulators (128 gate rows and
     // 128 up rows against one token tile) so a thread holds gate and up of its
     // feature; decode-width SwiGLU tiles split 64 gate + 64 up rows over the
     // lanes of one accumulator (more, smaller tiles for a short decode step).
-    constexpr bool kDual = MODE == kUpSwiglu && BN >= 64;
-    constexpr int kAStage = kDual ? 2 * kARows : kARows;
+    using C = Cfg<MODE, BN, WFMT, PAIR>;
+    static_assert(!(PAIR && WFMT), "SM pairs run bf16 weights");
+    constexpr bool kDual = C::kDual;
+    constexpr bool kInter = C::kInter;
+    constexpr int kAStage = C::kAStage;
     constexpr int kBoxRows = BN < 64 ? 16 : 64;       // token rows per TMA box
     // affine 4-bit: the A stage is written by the dequantisation warps from
     // packed codes (a quarter of the bf16 bytes) staged by TMA
-    constexpr int kCStage = WFMT ? kAStage / 4 : 0;
-    using L = Smem<BN, STAGES, kAStage, kCStage, MODE == kUpSwiglu && !kDual>;
+    constexpr int kCStage = C::kCStage;
+    using L = Smem<BN, STAGES, kAStage, kCStage, C::kHalves, (kCStage ? kSBDepth * 2 * kDq * 4 : 0), C::kBRows>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char* sA = sm + L::kA;
@@ -247,9 +275,12 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     int* s_off = s_cnt + 256;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;   // 0: the CTA that issues the pair's MMAs
     constexpr uint32_t kTmemCols = (kDual ? 4 : 2) * BN < 32 ? 32 : (kDual ? 4 : 2) * BN;
     // token rows come by TMA: from xs (up, gathered in plan order) or h (down)
-    constexpr uint32_t kFullCount = 1 + (WFMT ? 256 : 0);   // expect_tx arrive + 256 dequant threads
+    constexpr uint32_t kFullCount = 1 + (WFMT ? kDq : 0);   // expect_tx arrive + the dequant threads
+    // pairs: the even CTA's full barrier counts both CTAs' bytes (its producer
+    // arrives once with the total); its tempty barrier takes all 8 epilogue warps
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -259,19 +290,25 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], PAIR ? 8 : 4);
         }
         mbar_init(drain, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
+    if (PAIR) cluster_sync();     // both CTAs' barriers exist before either signals the other
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(s_tmem, kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(s_tmem, kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(s_tmem, kTmemCols);
+            tmem_relinquish();
+        }
         tc_fence_before();
     }
     // The up kernels follow the plan directly: they wait for it here.  The
@@ -286,8 +323,8 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     }
     __syncthreads();
     // tile table: tiles of expert e = weight tiles x ceil(count / BN)
-    const int fpt = (MODE == kUpSwiglu && !kDual) ? 64 : 128;   // output features per tile
-    const int n_wt = (g.feats + fpt - 1) / fpt;
+    const int fpt = C::kFpt;                                     // output features per tile (per CTA)
+    const int n_wt = (g.feats + fpt * (1 + PAIR) - 1) / (fpt * (1 + PAIR));   // weight tiles per expert
     if (warp == 2) {
         const int per = (g.E + 31) / 32;
         int local = 0;
@@ -319,6 +356,9 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     pdl_trigger();
     const uint32_t tmem_base = *s_tmem;
     const int nkb = g.K / kBK;
+    // the persistent tile loop: CTAs, or CTA pairs (both CTAs of a pair run the same tiles)
+    const int tbeg = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int tstep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
     // The down projection's scatter-add is linear, so its reduction can be
     // split: with less than ~4 waves of output tiles, K is cut into ks parts
     // (>= 4 k-blocks each) whose partial sums all add into y_acc.
@@ -326,7 +366,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     int ks = 1;
     if (kSplit && !g.ordered) {   // ordered: each slot row is stored once, whole
         const int t1 = max(s_base[g.E], 1);
-        ks = min(min(4, max(1, nkb / 4)), max(1, (4 * (int)gridDim.x + t1 - 1) / t1));
+        ks = min(min(4, max(1, nkb / 4)), max(1, (4 * tstep + t1 - 1) / t1));
     }
     const int total = s_base[g.E] * ks;
 
@@ -344,7 +384,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // down kernel: the first tile's first stages get their weight rows before
         // the wait on the up kernel; their token rows (h) follow after it
         int pre = 0;
-        if (MODE == kDown && blockIdx.x < total) {
+        if (MODE == kDown && !PAIR && blockIdx.x < total) {
             const Tile tl = decode_tile<BN, kSplit>(blockIdx.x, s_base, g.E, s_cnt, s_off, ks, nkb);
             pre = min(STAGES, tl.kb1 - tl.kb0);
             if (lane == 0) {
@@ -363,9 +403,12 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             }
         }
         if (MODE == kDown) pdl_wait();
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = tbeg; t < total && ok; t += tstep) {
             const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
-            const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt;
+            // pairs: this CTA's 128 weight rows of the 256-row tile, and its half of the token rows
+            const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt * (1 + PAIR) + (int)rank * fpt;
+            const int brows = PAIR ? tl.n / 2 : tl.n;
+            const int brow0 = tl.row0 + (int)rank * (PAIR ? tl.n / 2 : 0);
             for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 if (pre > 0) {
                     // weight rows already requested before the wait: add the token rows
@@ -384,7 +427,19 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 // all 32 lanes wait on the same phase; the decision is made warp-uniform
                 const bool got = mbar_wait(&empty[s], ph ^ 1, s_abort, g.wait_limit);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-                if (lane == 0) {
+                if (lane == 0 && PAIR) {
+                    // both CTAs' loads complete on the even CTA's full barrier; it arrives once
+                    // with the bytes of both
+                    const int nbox = (brows + kBoxRows - 1) / kBoxRows;
+                    const uint32_t fb = mapa_shared(smem_u32(&full[s]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2u * (kAStage + nbox * kBoxRows * 128));
+                    unsigned char* a = sA + size_t(s) * kAStage;
+                    tma_load_2d_pair(a, &tmA, kb * kBK, a_row, fb);
+                    if (MODE == kUpSwiglu) tma_load_2d_pair(a + kAStage / 2, &tmA, kb * kBK, a_row + g.I, fb);
+                    unsigned char* b = sB + size_t(s) * L::kBStage;
+                    for (int j = 0; j < nbox; ++j)
+                        tma_load_2d_pair(b + j * kBoxRows * 128, &tmB, kb * kBK, brow0 + kBoxRows * j, fb);
+                } else if (lane == 0) {
                     const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
                     const uint32_t bytes = (WFMT ? 0 : kAStage) + nbox * kBoxRows * 128;
                     mbar_arrive_expect_tx(&full[s], bytes);
@@ -416,23 +471,27 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             *s_abort = 1;
         }
         // wait (bounded) for every fill this warp issued to land before the CTA can exit
-        for (int q = 0; q < STAGES; ++q)
-            if (issued_mask >> q & 1u) mbar_wait(&full[q], issued_par >> q & 1u, nullptr, g.wait_limit);
+        // (pairs: the even CTA's full barriers count the odd CTA's bytes too, and the
+        // two CTAs meet at a cluster barrier before either exits)
+        if (!PAIR || rank == 0)
+            for (int q = 0; q < STAGES; ++q)
+                if (issued_mask >> q & 1u) mbar_wait(&full[q], issued_par >> q & 1u, nullptr, g.wait_limit);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // (pairs: only the even CTA issues; its MMAs cover both CTAs' rows)
+        if (lane == 0 && rank == 0) {
             int s = 0;
             uint32_t ph = 0;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+            for (int t = tbeg; t < total && ok; t += tstep, ++it) {
                 const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
                 const int buf = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort, g.wait_limit)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * (kDual ? 2 * BN : BN);
-                const uint32_t idesc = idesc_bf16(128, tl.n);
+                const uint32_t idesc = idesc_bf16(PAIR ? 256 : 128, tl.n);
                 for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                     if (!mbar_wait(&full[s], ph, s_abort, g.wait_limit)) { ok = false; break; }
                     tc_fence_after();
@@ -440,48 +499,66 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     const uint64_t bd = sdesc_sw128(smem_u32(sB + size_t(s) * L::kBStage));
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
-                        umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, kb != tl.kb0 || kk != 0);
-                        if (kDual)   // up rows: the second 16 KB of the A stage, accumulator at + BN columns
-                            umma_bf16(d + BN, ad + uint64_t((kARows >> 4) + kk * 2), bd + uint64_t(kk * 2), idesc,
-                                      kb != tl.kb0 || kk != 0);
+                        const bool acc = kb != tl.kb0 || kk != 0;
+                        if (PAIR) {
+                            umma_bf16_pair(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, acc);
+                            if (kDual)
+                                umma_bf16_pair(d + BN, ad + uint64_t((kARows >> 4) + kk * 2), bd + uint64_t(kk * 2),
+                                               idesc, acc);
+                        } else {
+                            umma_bf16(d, ad + uint64_t(kk * 2), bd + uint64_t(kk * 2), idesc, acc);
+                            if (kDual)   // up rows: the second 16 KB of the A stage, accumulator at + BN columns
+                                umma_bf16(d + BN, ad + uint64_t((kARows >> 4) + kk * 2), bd + uint64_t(kk * 2), idesc,
+                                          acc);
+                        }
                     }
-                    umma_commit(&empty[s]);
+                    if (PAIR) umma_commit_pair_both(&empty[s]);   // both CTAs' stage s is free again
+                    else umma_commit(&empty[s]);
                     if (++s == STAGES) { s = 0; ph ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(&tfull[buf]);
+                if (PAIR) umma_commit_pair_both(&tfull[buf]);      // both CTAs' accumulators are ready
+                else umma_commit(&tfull[buf]);
             }
             if (!ok) {
                 report_error(g.err, kErrWaitExpired);
                 *s_abort = 1;
             }
             // all MMAs issued by this thread complete before TMEM is freed
-            umma_commit(drain);
+            if (PAIR) umma_commit_pair_local(drain);
+            else umma_commit(drain);
             mbar_wait(drain, 0, nullptr, g.wait_limit);
         }
         __syncwarp();
-    } else if (WFMT && warp >= 6) {   // warps 6..13
-        // ------------------------------------------------------------ dequantisation (affine 4-bit)
-        // 256 threads.  Thread dt owns A row r (two threads per row at decode
-        // width, each half of its 8 chunks).  Each thread fetches its row's
-        // scale and bias kSBDepth stages ahead with 4-byte cp.async into a ring
-        // in shared memory (the word holding the bf16; the half is picked later).
+    } else if (WFMT && warp >= 6) {   // warps 6 .. 6 + kDq / 32 - 1
+        // ------------------------------------------------------------ dequantisation (4-bit)
+        // kDq threads.  kTpr threads share an A row, each kCPT of its 8 chunks.
+        // Each thread fetches its row's scale (and bias) kSBDepth stages ahead
+        // with 4-byte cp.async into a ring in shared memory (affine: the word
+        // holding the bf16, the half is picked later; NVFP4: the row's four
+        // e4m3 block scales of the k-block).
         const int dt = threadIdx.x - 192;
-        constexpr int kCPT = kDual ? 8 : 4;
-        const int r = kDual ? dt : (dt >> 1);
-        const int cbeg = kDual ? 0 : (dt & 1) * 4;
+        constexpr int kRows = kDual ? 256 : 128;
+        constexpr int kTpr = kDq / kRows;                  // threads per A row
+        constexpr int kCPT = 8 / kTpr;                     // 16-byte chunks per thread
+        const int r = dt / kTpr;
+        const int cbeg = (dt % kTpr) * kCPT;
         const int halfr = kDual ? 128 : 64;                // SwiGLU: rows of the gate half
         const size_t nrows = (size_t)g.E_w * g.rows_per_expert;
         const int G = g.K / 64;
         uint32_t* s_sb = reinterpret_cast<uint32_t*>(sm + L::kSB);
+        // inter layout: A row r = 32 q + j holds gate (j < 16) or up (j >= 16) of
+        // feature 16 q + (j & 15) of the tile; the staged codes are 64 gate rows
+        // then 64 up rows, as TMA brings them
+        const int cr = kInter ? ((r & 16) ? 64 : 0) + 16 * (r >> 5) + (r & 15) : r;   // staged code row
         auto grow = [&](const Tile& tl) -> size_t {      // global weight row of A row r
             const size_t base = (size_t)tl.e * g.rows_per_expert;
             if (MODE == kUpSwiglu)
-                return r < halfr ? base + (size_t)tl.wt * halfr + r : base + g.I + (size_t)tl.wt * halfr + (r - halfr);
+                return cr < halfr ? base + (size_t)tl.wt * halfr + cr : base + g.I + (size_t)tl.wt * halfr + (cr - halfr);
             return base + (size_t)tl.wt * 128 + r;
         };
         // look-ahead iterator over this CTA's (tile, k-block) stages
-        int at = blockIdx.x, akb = 0;
+        int at = tbeg, akb = 0;
         Tile atl{};
         if (at < total) {
             atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
@@ -492,15 +569,15 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 const size_t gr = grow(atl);
                 if (WFMT == 2) {      // the row's four e4m3 block scales of this k-block: one word
                     const size_t wi = gr < nrows ? gr * (size_t)(g.K / 16) + 4 * (size_t)akb : 0;
-                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt),
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * kDq + dt),
                               reinterpret_cast<const uint8_t*>(g.wscale) + wi);
                 } else {
                     const size_t gi = gr < nrows ? gr * G + akb : 0;
-                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * 256 + dt), g.wscale + (gi & ~size_t(1)));
-                    cp_async4(smem_u32(s_sb + (slot * 2 + 1) * 256 + dt), g.wbias + (gi & ~size_t(1)));
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 0) * kDq + dt), g.wscale + (gi & ~size_t(1)));
+                    cp_async4(smem_u32(s_sb + (slot * 2 + 1) * kDq + dt), g.wbias + (gi & ~size_t(1)));
                 }
                 if (++akb == atl.kb1) {
-                    at += gridDim.x;
+                    at += tstep;
                     if (at < total) {
                         atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
                         akb = atl.kb0;
@@ -514,13 +591,13 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int s = 0, slot = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = tbeg; t < total && ok; t += tstep) {
             const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
             const size_t gr = grow(tl);
             for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 cp_async_wait<kSBDepth - 1>();               // this stage's scale/bias landed
-                const uint32_t sw = s_sb[(slot * 2 + 0) * 256 + dt];
-                const uint32_t bw = s_sb[(slot * 2 + 1) * 256 + dt];
+                const uint32_t sw = s_sb[(slot * 2 + 0) * kDq + dt];
+                const uint32_t bw = s_sb[(slot * 2 + 1) * kDq + dt];
                 const bool odd = ((gr * G + kb) & 1) != 0;
                 const bool inb = gr < nrows;
                 const uint16_t sc = inb ? uint16_t(odd ? sw >> 16 : sw & 0xFFFFu) : uint16_t(0);
@@ -528,15 +605,24 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 issue(slot);                                  // refill the slot kSBDepth stages ahead
                 if (++slot == kSBDepth) slot = 0;
                 if (!mbar_wait(&cfull[s], ph, s_abort, g.wait_limit)) { ok = false; break; }
-                const uint32_t* crow = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage) + r * 8 + cbeg;
+                const uint32_t* crow = reinterpret_cast<const uint32_t*>(sC + size_t(s) * kCStage) + cr * 8 + cbeg;
                 uint32_t cw[kCPT];
+                if (kCPT >= 4) {
 #pragma unroll
-                for (int q = 0; q < kCPT / 4; ++q) {
-                    const uint4 c4 = reinterpret_cast<const uint4*>(crow)[q];
-                    cw[4 * q + 0] = c4.x;
-                    cw[4 * q + 1] = c4.y;
-                    cw[4 * q + 2] = c4.z;
-                    cw[4 * q + 3] = c4.w;
+                    for (int q = 0; q < kCPT / 4; ++q) {
+                        const uint4 c4 = reinterpret_cast<const uint4*>(crow)[q];
+                        cw[4 * q + 0] = c4.x;
+                        cw[4 * q + 1] = c4.y;
+                        cw[4 * q + 2] = c4.z;
+                        cw[4 * q + 3] = c4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < kCPT / 2; ++q) {
+                        const uint2 c2 = reinterpret_cast<const uint2*>(crow)[q];
+                        cw[2 * q + 0] = c2.x;
+                        cw[2 * q + 1] = c2.y;
+                    }
                 }
                 if (WFMT == 2)
                     dequant_nvfp4_chunks<kCPT>(cw, cbeg, inb ? sw : 0u, sA + size_t(s) * kAStage + r * 128, r);
@@ -562,10 +648,11 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         const int et = threadIdx.x - 64;          // 0..127
         int it = 0;
         bool dead = false;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+        for (int t = tbeg; t < total; t += tstep, ++it) {
             const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
             const int buf = it & 1;
             const uint32_t aph = (it >> 1) & 1;
+            const int fbase = tl.wt * fpt * (1 + PAIR) + (int)rank * fpt;   // first output feature of this CTA
             if (MODE == kDown) {
                 for (int c = et; c < tl.ntok; c += 128) {
                     const int p = g.perm[tl.row0 + c];
@@ -598,7 +685,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     }
                 }
                 if (MODE == kDown) {
-                    const int f = tl.wt * 128 + lrow;
+                    const int f = fbase + lrow;
                     if (!dead && f < g.feats) {
                         if (!g.ordered) {
 #pragma unroll
@@ -615,12 +702,35 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                         }
                     }
                 } else if (MODE == kUpRelu2) {
-                    const int f = tl.wt * 128 + lrow;
+                    const int f = fbase + lrow;
                     if (!dead && f < g.feats) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
                             if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_relu2(v[i]));
+                        }
+                    }
+                } else if (kInter) {
+                    // lanes 0-15: gate of feature f, lanes 16-31: up of f (f = 16 sub + lane % 16
+                    // within the tile).  One exchange of eight values: the low lanes then
+                    // hold gate and up of columns c0 .. c0+7, the high lanes of c0+8 .. c0+15.
+                    const bool lo = lane < 16;
+                    const int f = fbase + 16 * sub + (lane & 15);
+                    float gv[8], uv[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float other = __shfl_xor_sync(0xffffffffu, lo ? v[8 + i] : v[i], 16);
+                        gv[i] = lo ? v[i] : other;
+                        uv[i] = lo ? other : v[8 + i];
+                    }
+                    if (!dead && f < g.feats) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int c = c0 + (lo ? i : 8 + i);
+                            if (c >= tl.ntok) continue;
+                            float a_ = gv[i], b_ = uv[i];
+                            clamp_swiglu(a_, b_, g.swiglu_limit);
+                            g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(a_, b_));
                         }
                     }
                 } else if (kDual) {
@@ -635,7 +745,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                             for (int i = 0; i < 16; ++i) u[i] *= gsc;
                         }
                     }
-                    const int f = tl.wt * 128 + lrow;
+                    const int f = fbase + lrow;
                     if (!dead && f < g.feats) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -654,7 +764,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     }
                     named_bar(1, 128);
                     if (!dead && sub < 2) {
-                        const int f = tl.wt * 64 + lrow;
+                        const int f = fbase + lrow;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int c = c0 + i;
@@ -668,14 +778,19 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 }
             }
             tc_fence_before();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
+            if (lane == 0) {
+                if (PAIR && rank != 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+                else mbar_arrive(&tempty[buf]);
+            }
             if (MODE == kDown) named_bar(1, 128);   // s_tok reuse
         }
     }
     __syncthreads();
+    if (PAIR) cluster_sync();     // the pair's MMAs and both epilogues are done with TMEM
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+        else tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
@@ -729,10 +844,11 @@ cudaError_t make_tmap_u32(CUtensorMap* m, const void* base, uint64_t inner, uint
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int MODE, int BN, int STAGES, int WFMT>
+template <int MODE, int BN, int STAGES, int WFMT, int PAIR = 0>
 cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, bool pdl, cudaStream_t s) {
     CUtensorMap tA, tB;
-    const uint32_t a_box = (MODE == kUpSwiglu && BN < 64) ? 64 : 128;
+    using C = Cfg<MODE, BN, WFMT, PAIR>;
+    const uint32_t a_box = C::kABox;
     const uint32_t b_box = BN < 64 ? 16 : 64;
     cudaError_t e;
     if (WFMT)   // 8 code words (64 codes) of one k-block per row
@@ -746,12 +862,14 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
         e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, b_box);   // rows gathered in plan order
     }
     if (e != cudaSuccess) return e;
-    auto kern = k_gemm<MODE, BN, STAGES, WFMT>;
-    constexpr int kA = (MODE == kUpSwiglu && BN >= 64) ? 2 * kARows : kARows;
-    using L = Smem<BN, STAGES, kA, WFMT ? kA / 4 : 0, MODE == kUpSwiglu && BN < 64>;   // + scale/bias ring (affine)
+    auto kern = k_gemm<MODE, BN, STAGES, WFMT, PAIR>;
+    using L = Smem<BN, STAGES, C::kAStage, C::kCStage, C::kHalves, (C::kCStage ? kSBDepth * 2 * kDq * 4 : 0),
+                   C::kBRows>;   // the kernel's own layout
     static_assert(L::kBytes <= 227 * 1024, "shared memory of one CTA");
     const size_t smem = L::kBytes;
     if ((e = ensure_smem(kern, smem)) != cudaSuccess) return e;
+    if (PAIR)   // one CTA per SM, in pairs on neighbouring SMs
+        return launch_k_pair(kern, dim3(device_info().sm_count & ~1), dim3(kThreads), smem, s, pdl, tA, tB, g);
     return launch_k(kern, dim3(device_info().sm_count), dim3(WFMT ? kThreadsA4 : kThreads), smem, s, pdl, tA,
                     tB, g);
 }
@@ -832,7 +950,8 @@ template <int WFMT>
 cudaError_t gemm_up_q4(const ExpertArgs& a, const GemmParams& g, int bn, bool pdl, cudaStream_t s) {
     if (a.act == 0) {
         if (bn == 32) return run<kUpSwiglu, 32, 8, WFMT>(a, g, a.w1, pdl, s);
-        return run<kUpSwiglu, 128, 3, WFMT>(a, g, a.w1, pdl, s);
+        if (bn == 128) return run<kUpSwiglu, 128, 5, WFMT>(a, g, a.w1, pdl, s);   // inter layout
+        return run<kUpSwiglu, 256, 3, WFMT>(a, g, a.w1, pdl, s);                   // inter layout, 256 tokens
     }
     if (bn == 32) return run<kUpRelu2, 32, 8, WFMT>(a, g, a.w1, pdl, s);
     if (bn == 128) return run<kUpRelu2, 128, 5, WFMT>(a, g, a.w1, pdl, s);
@@ -852,13 +971,16 @@ cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const GemmParams g = params(a, true);
     const int bn = pick_bn(a);
     if (a.fmt == 0) {
+        // token tiles of 128 and more: M = 256 tiles on SM pairs
         if (a.act == 0) {
+            // bf16 SwiGLU keeps one CTA per tile with two accumulators: measured
+            // faster in the benchmark loop than either layout on SM pairs
             if (bn == 32) return run<kUpSwiglu, 32, 8, 0>(a, g, a.w1, pdl, s);
             return run<kUpSwiglu, 128, 4, 0>(a, g, a.w1, pdl, s);   // two accumulators: 4 x 128 TMEM columns
         }
         if (bn == 32) return run<kUpRelu2, 32, 8, 0>(a, g, a.w1, pdl, s);
-        if (bn == 128) return run<kUpRelu2, 128, 5, 0>(a, g, a.w1, pdl, s);
-        return run<kUpRelu2, 256, 4, 0>(a, g, a.w1, pdl, s);
+        if (bn == 128) return run<kUpRelu2, 128, 8, 0, 1>(a, g, a.w1, pdl, s);
+        return run<kUpRelu2, 256, 6, 0, 1>(a, g, a.w1, pdl, s);
     }
     if (a.fmt == 1) return gemm_up_q4<1>(a, g, bn, pdl, s);
     if (a.fmt == 2) return gemm_up_q4<2>(a, g, bn, pdl, s);
@@ -870,8 +992,8 @@ cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const int bn = pick_bn(a);
     if (a.fmt == 0) {
         if (bn == 32) return run<kDown, 32, 8, 0>(a, g, a.w2, pdl, s);
-        if (bn == 128) return run<kDown, 128, 5, 0>(a, g, a.w2, pdl, s);
-        return run<kDown, 256, 4, 0>(a, g, a.w2, pdl, s);
+        if (bn == 128) return run<kDown, 128, 8, 0, 1>(a, g, a.w2, pdl, s);
+        return run<kDown, 256, 6, 0, 1>(a, g, a.w2, pdl, s);
     }
     if (a.fmt == 1) return gemm_down_q4<1>(a, g, bn, pdl, s);
     if (a.fmt == 2) return gemm_down_q4<2>(a, g, bn, pdl, s);

@@ -29,8 +29,9 @@
 // with each 8-k group reordered (x0 x4 x1 x5 x2 x6 x3 x7) to match, so the B
 // fragments load straight from shared memory.  Per group of 64 k and row,
 //     sum_k w x = s * sum_k (128 + q) x + (b - 128 s) * sum_k x,
-// with sum_k x precomputed per token and group at staging, and the group's
-// scale and bias staged per unit in shared memory.
+// with sum_k x precomputed per token and group at staging; the group's scale
+// and bias ride in the code ring (lane tq of a quad fetches one of the four
+// values its quad needs, and shuffles share them).
 //
 // NVFP4 (f16 MMA): cvt.rn.f16x2.e2m1x2 turns a code byte into an f16 pair and
 // one f16 multiply by the block scale gives e2m1 * e4m3 exactly (at most six
@@ -111,17 +112,15 @@ MOE_DEV uint32_t ld_u8(const uint8_t* p) {
 MOE_DEV __host__ int q_stride(int K) { return K + 8; }
 
 struct QLayout {          // dynamic shared memory of one CTA (byte offsets)
-    int x, sx, sb, total;
+    int x, sx, total;
 };
 
-MOE_DEV __host__ QLayout q_layout(int fmt, int K, int rows_cta) {
+MOE_DEV __host__ QLayout q_layout(int fmt, int K) {
     QLayout L;
     L.x = 0;
     int off = kQTok * q_stride(K) * 2;
     L.sx = off;                                   // affine: sum_k x per (group, token), [G][8] fp32
     if (fmt == kQAffine) off += (K / 64) * kQTok * 4;
-    L.sb = off;                                   // affine: (scale | bias << 16) per (row, group), stride G + 1
-    if (fmt == kQAffine) off += rows_cta * (K / 64 + 1) * 4;
     L.total = off;
     return L;
 }
@@ -143,10 +142,9 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
     const int RB = MODE == kQUpSwiglu ? a.I / 8 : N / 16;              // MMA row blocks per expert
     const int NRQ = (RB + RBC - 1) / RBC;                              // row blocks of a CTA
     const int XS = q_stride(K);
-    const QLayout L = q_layout(FMT, K, RBC * 16);
+    const QLayout L = q_layout(FMT, K);
     uint16_t* s_x = reinterpret_cast<uint16_t*>(q_smem + L.x);
     float* s_sx = reinterpret_cast<float*>(q_smem + L.sx);
-    uint32_t* s_sb = reinterpret_cast<uint32_t*>(q_smem + L.sb);
     const uint8_t* codes = reinterpret_cast<const uint8_t*>(down ? a.w2 : a.w1);
     const uint16_t* wsc = down ? a.w2_scale : a.w1_scale;   // affine scale (bf16) / NVFP4 e4m3 bytes
     const uint16_t* wbi = down ? a.w2_bias : a.w1_bias;     // affine bias
@@ -178,6 +176,8 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
     const int nsteps = KW / kQStepK;
     const int rbl = warp / KS, ks = warp % KS;
     const int kbeg = ks * KW;
+    // affine: lane tq of a quad fetches one of (scale row g, bias row g, scale row g+8, bias row g+8)
+    const uint16_t* sbsrc = tq & 1 ? wbi : wsc;
 
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
         int lo = 0, hi = a.E;                    // expert: last e with s_base[e] <= u
@@ -217,6 +217,7 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
                     q0[d] = ld_codes(p0 + 32 * d, pol);
                     q1[d] = ld_codes(p1 + 32 * d, pol);
                     if (FMT == kQNvfp4) sc[d] = ld_u8(ps0 + 4 * d) | (ld_u8(ps1 + 4 * d) << 8);
+                    else sc[d] = __ldg(sbsrc + (tq < 2 ? r0 : r1) * G + kbeg / 64 + d);
                 }
             }
         }
@@ -278,26 +279,11 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
                 }
             }
         }
-        if (FMT == kQAffine) {                   // the unit's rows' scale and bias, every group
-            const int nrow = RBC * 16, GS = G + 1;
-            for (int i = threadIdx.x; i < nrow * G; i += blockDim.x) {
-                const int rl = i / G, gi = i - rl * G;
-                const int b = rq * RBC + rl / 16;
-                uint32_t v = 0;
-                if (b < RB) {
-                    const size_t gidx = (ebase + wrow(b, rl % 16)) * G + gi;
-                    v = uint32_t(__ldg(wsc + gidx)) | (uint32_t(__ldg(wbi + gidx)) << 16);
-                }
-                s_sb[rl * GS + gi] = v;
-            }
-        }
         __syncthreads();
 
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         if (active) {
             const uint16_t* xr = s_x + g * XS + kbeg + 16 * tq;
-            const uint32_t* sbr0 = s_sb + (rbl * 16 + g) * (G + 1) + kbeg / 64;
-            const uint32_t* sbr1 = s_sb + (rbl * 16 + g + 8) * (G + 1) + kbeg / 64;
             for (int sb = 0; sb < nsteps; sb += kQRing) {
 #pragma unroll
                 for (int d = 0; d < kQRing; ++d) {
@@ -334,9 +320,12 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
                                 mma_bf16_16816(cg, nib_pair(v, 2), nib_pair(w, 2), nib_pair(v, 3), nib_pair(w, 3),
                                                xv.z, xv.w);
                             }
-                            const uint32_t b0 = sbr0[st], b1 = sbr1[st];
-                            const float s0 = bf16lo(b0), s1 = bf16lo(b1);
-                            const float c0 = fmaf(-128.f, s0, bf16hi(b0)), c1 = fmaf(-128.f, s1, bf16hi(b1));  // exact
+                            const int qb = lane & ~3;
+                            const float s0 = bf16f((uint16_t)__shfl_sync(0xffffffffu, sc[d], qb + 0));
+                            const float b0 = bf16f((uint16_t)__shfl_sync(0xffffffffu, sc[d], qb + 1));
+                            const float s1 = bf16f((uint16_t)__shfl_sync(0xffffffffu, sc[d], qb + 2));
+                            const float b1 = bf16f((uint16_t)__shfl_sync(0xffffffffu, sc[d], qb + 3));
+                            const float c0 = fmaf(-128.f, s0, b0), c1 = fmaf(-128.f, s1, b1);   // exact
                             const float2 sx = *reinterpret_cast<const float2*>(s_sx + (kbeg / 64 + st) * kQTok + 2 * tq);
                             acc[0] = fmaf(s0, cg[0], fmaf(c0, sx.x, acc[0]));
                             acc[1] = fmaf(s0, cg[1], fmaf(c0, sx.y, acc[1]));
@@ -348,6 +337,8 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
                             q1[d] = ld_codes(p1 + 32 * (st + kQRing), pol);
                             if (FMT == kQNvfp4)
                                 sc[d] = ld_u8(ps0 + 4 * (st + kQRing)) | (ld_u8(ps1 + 4 * (st + kQRing)) << 8);
+                            else
+                                sc[d] = __ldg(sbsrc + (tq < 2 ? r0 : r1) * G + kbeg / 64 + st + kQRing);
                         }
                     }
                 }
@@ -399,7 +390,7 @@ __global__ void __launch_bounds__(kQWarps * 32, 2) k_gemv_q4(ExpertArgs a) {
                 }
             }
         }
-        __syncthreads();                         // s_x, s_sb, s_tm and s_red are rewritten by the next unit
+        __syncthreads();                         // s_x, s_sx, s_tm and s_red are rewritten by the next unit
     }
     pdl_trigger();
 }
@@ -422,7 +413,7 @@ int q_choose_ks(const ExpertArgs& a, int K, int RB) {
 
 template <int FMT, int MODE, int KS>
 cudaError_t run_q4(const ExpertArgs& a, int K, bool pdl, cudaStream_t s) {
-    const QLayout L = q_layout(FMT, K, (kQWarps / KS) * 16);
+    const QLayout L = q_layout(FMT, K);
     auto kern = k_gemv_q4<FMT, MODE, KS>;
     cudaError_t e = ensure_smem(kern, (size_t)L.total);
     if (e != cudaSuccess) return e;
