@@ -537,6 +537,9 @@ class Runner:
             if sid == abi.MOE_STAGE_GATHER and gemv_path:
                 out[nm] = "not launched (GEMV path)"
                 continue
+            if sid == abi.MOE_STAGE_GATHER and self.wl.fmt == "bf16" and self.wl.T <= 16:
+                out[nm] = "not launched (the up GEMM reads x itself at T <= 16)"
+                continue
             evs = self._events(B)
             self.stream.synchronize()
             g = torch.cuda.CUDAGraph()
@@ -561,7 +564,7 @@ def dtype_of(wl) -> str:
 
 
 def gemv_path_of(wl, dispatch: str) -> bool:
-    """The library's AUTO choice: affine 4-bit experts at <= 8 pairs per expert take the GEMV."""
+    """The library's AUTO choice: 4-bit experts at <= 8 pairs per expert take the GEMV."""
     return dispatch == "gemv" or (dispatch == "auto" and wl.fmt != "bf16" and wl.T * wl.k <= 8 * wl.E
                                   and wl.H <= 8192 and wl.I <= 8192)
 

@@ -54,6 +54,17 @@ MOE_DEV uint64_t policy_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+MOE_DEV uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 16-byte store with an L2 eviction policy (a buffer the next kernel re-reads)
+MOE_DEV void st_hint(void* p, uint4 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1,%2,%3,%4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w), "l"(policy)
+                 : "memory");
+}
 // Read-only 16-byte load that may stay in L1 (activations reused across rows).
 MOE_DEV uint4 ld_nc(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 

@@ -43,6 +43,7 @@
 #include "plan_dev.cuh"
 #include "quant.cuh"
 #include "sm100.cuh"
+#include "tmap.h"
 
 namespace moe {
 namespace {
@@ -78,6 +79,9 @@ struct GemmParams {
     int skip;                // plan expert given no tiles (its pairs are computed nowhere), or -1
     int E_w;                 // experts the weight tensor holds
     uint32_t wait_limit;     // polls of every bounded pipeline wait (sm100::kWaitLimit)
+    int dense_n;             // bf16 up at T <= 16: the token operand is x itself (rows 0..T-1, the
+                             // MMA's N = dense_n = T rounded up to 16) and column t is token t;
+                             // 0: token rows gathered in plan order (xs), column c is slot row0 + c
     int* err;
 };
 
@@ -127,6 +131,7 @@ struct Cfg {
 
 struct Tile {
     int e, wt, tt, ntok, n, row0;
+    int brow;                // first token row the TMA reads (row0, or 0 when the operand is x)
     int kb0, kb1;            // k-blocks of this tile (a part of K when the reduction is split)
 };
 
@@ -136,7 +141,8 @@ struct Tile {
 // With SPLIT, ks consecutive tile numbers share one output tile and each
 // takes a contiguous part of the nkb k-blocks.
 template <int BN, bool SPLIT>
-MOE_DEV Tile decode_tile(int tn, const int* base, int E, const int* counts, const int* offsets, int ks, int nkb) {
+MOE_DEV Tile decode_tile(int tn, const int* base, int E, const int* counts, const int* offsets, int ks, int nkb,
+                         int dense_n) {
     const int t = SPLIT ? tn / ks : tn;
     int lo = 0, hi = E;
     while (lo < hi) {
@@ -154,6 +160,11 @@ MOE_DEV Tile decode_tile(int tn, const int* base, int E, const int* counts, cons
     r.ntok = min(BN, c - r.tt * BN);
     r.n = (r.ntok + 15) & ~15;
     r.row0 = offsets[lo] + r.tt * BN;
+    r.brow = r.row0;
+    if (dense_n) {
+        r.n = dense_n;
+        r.brow = 0;
+    }
     if (SPLIT) {
         const int part = tn - t * ks;
         r.kb0 = part * nkb / ks;
@@ -324,6 +335,8 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
     __syncthreads();
     // tile table: tiles of expert e = weight tiles x ceil(count / BN)
     const int fpt = C::kFpt;                                     // output features per tile (per CTA)
+    constexpr bool kDenseOk = MODE != kDown && BN == 32 && WFMT == 0 && !PAIR;
+    const int dense_n = kDenseOk ? g.dense_n : 0;                // token operand = x (see GemmParams)
     const int n_wt = (g.feats + fpt * (1 + PAIR) - 1) / (fpt * (1 + PAIR));   // weight tiles per expert
     if (warp == 2) {
         const int per = (g.E + 31) / 32;
@@ -385,7 +398,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         // the wait on the up kernel; their token rows (h) follow after it
         int pre = 0;
         if (MODE == kDown && !PAIR && blockIdx.x < total) {
-            const Tile tl = decode_tile<BN, kSplit>(blockIdx.x, s_base, g.E, s_cnt, s_off, ks, nkb);
+            const Tile tl = decode_tile<BN, kSplit>(blockIdx.x, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
             pre = min(STAGES, tl.kb1 - tl.kb0);
             if (lane == 0) {
                 const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
@@ -404,11 +417,11 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         }
         if (MODE == kDown) pdl_wait();
         for (int t = tbeg; t < total && ok; t += tstep) {
-            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
             // pairs: this CTA's 128 weight rows of the 256-row tile, and its half of the token rows
             const int a_row = tl.e * g.rows_per_expert + tl.wt * fpt * (1 + PAIR) + (int)rank * fpt;
             const int brows = PAIR ? tl.n / 2 : tl.n;
-            const int brow0 = tl.row0 + (int)rank * (PAIR ? tl.n / 2 : 0);
+            const int brow0 = tl.brow + (int)rank * (PAIR ? tl.n / 2 : 0);
             for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 if (pre > 0) {
                     // weight rows already requested before the wait: add the token rows
@@ -416,7 +429,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                         const int nbox = (tl.n + kBoxRows - 1) / kBoxRows;
                         unsigned char* b = sB + size_t(s) * L::kBStage;
                         for (int j = 0; j < nbox; ++j)
-                            tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
+                            tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.brow + kBoxRows * j, &full[s]);
                     }
                     --pre;
                     issued_mask |= 1u << s;
@@ -459,7 +472,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     }
                     unsigned char* b = sB + size_t(s) * L::kBStage;
                     for (int j = 0; j < nbox; ++j)
-                        tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.row0 + kBoxRows * j, &full[s]);
+                        tma_load_2d(b + j * kBoxRows * 128, &tmB, kb * kBK, tl.brow + kBoxRows * j, &full[s]);
                 }
                 issued_mask |= 1u << s;
                 issued_par = (issued_par & ~(1u << s)) | (ph << s);
@@ -485,7 +498,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = tbeg; t < total && ok; t += tstep, ++it) {
-                const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
+                const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
                 const int buf = it & 1;
                 const uint32_t aph = (it >> 1) & 1;
                 if (!mbar_wait(&tempty[buf], aph ^ 1, s_abort, g.wait_limit)) { ok = false; break; }
@@ -561,7 +574,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int at = tbeg, akb = 0;
         Tile atl{};
         if (at < total) {
-            atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
+            atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
             akb = atl.kb0;
         }
         auto issue = [&](int slot) {
@@ -579,7 +592,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 if (++akb == atl.kb1) {
                     at += tstep;
                     if (at < total) {
-                        atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb);
+                        atl = decode_tile<BN, kSplit>(at, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
                         akb = atl.kb0;
                     }
                 }
@@ -592,7 +605,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         uint32_t ph = 0;
         bool ok = true;
         for (int t = tbeg; t < total && ok; t += tstep) {
-            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
             const size_t gr = grow(tl);
             for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
                 cp_async_wait<kSBDepth - 1>();               // this stage's scale/bias landed
@@ -649,7 +662,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
         int it = 0;
         bool dead = false;
         for (int t = tbeg; t < total; t += tstep, ++it) {
-            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb);
+            const Tile tl = decode_tile<BN, kSplit>(t, s_base, g.E, s_cnt, s_off, ks, nkb, dense_n);
             const int buf = it & 1;
             const uint32_t aph = (it >> 1) & 1;
             const int fbase = tl.wt * fpt * (1 + PAIR) + (int)rank * fpt;   // first output feature of this CTA
@@ -660,7 +673,18 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     s_tokw[c] = g.topk_w[p];
                 }
                 named_bar(1, 128);
+            } else if (dense_n) {
+                // column t is token t: its h row is the plan slot of (t, this expert), if routed here
+                for (int c = et; c < tl.n; c += 128) s_tok[c] = -1;
+                named_bar(1, 128);
+                for (int c = et; c < tl.ntok; c += 128) s_tok[g.perm[tl.row0 + c] / g.k] = tl.row0 + c;
+                named_bar(1, 128);
             }
+            // h row of accumulator column c (up), or -1
+            auto hrow = [&](int c) -> int {
+                if (dense_n) return s_tok[c];
+                return c < tl.ntok ? tl.row0 + c : -1;
+            };
             if (!dead) {
                 const bool ok = mbar_wait(&tfull[buf], aph, s_abort, g.wait_limit);
                 if (__any_sync(0xffffffffu, !ok)) {     // warp-uniform: tcgen05.ld is warp-collective
@@ -706,8 +730,8 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                     if (!dead && f < g.feats) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const int c = c0 + i;
-                            if (c < tl.ntok) g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(act_relu2(v[i]));
+                            const int r = hrow(c0 + i);
+                            if (r >= 0) g.h[(size_t)r * g.I + f] = f2bf16(act_relu2(v[i]));
                         }
                     }
                 } else if (kInter) {
@@ -767,11 +791,11 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                         const int f = fbase + lrow;
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const int c = c0 + i;
-                            if (c >= tl.ntok) continue;
+                            const int r = hrow(c0 + i);
+                            if (r < 0) continue;
                             float gv = v[i], uv = s_u[lrow * 17 + i];
                             clamp_swiglu(gv, uv, g.swiglu_limit);
-                            g.h[(size_t)(tl.row0 + c) * g.I + f] = f2bf16(silu_mul(gv, uv));
+                            g.h[(size_t)r * g.I + f] = f2bf16(silu_mul(gv, uv));
                         }
                     }
                     named_bar(1, 128);
@@ -782,7 +806,7 @@ __global__ void __launch_bounds__(WFMT ? kThreadsA4 : kThreads, 1)
                 if (PAIR && rank != 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
                 else mbar_arrive(&tempty[buf]);
             }
-            if (MODE == kDown) named_bar(1, 128);   // s_tok reuse
+            if (MODE == kDown || dense_n) named_bar(1, 128);   // s_tok reuse
         }
     }
     __syncthreads();
@@ -858,6 +882,8 @@ cudaError_t run(const ExpertArgs& a, const GemmParams& g, const void* wbase, boo
     if (e != cudaSuccess) return e;
     if (MODE == kDown) {
         e = make_tmap(&tB, a.h, (uint64_t)a.I, (uint64_t)a.T * a.k, kBK, b_box);
+    } else if (g.dense_n) {
+        e = make_tmap(&tB, a.x, (uint64_t)a.H, (uint64_t)a.T, kBK, b_box);          // x itself, rows 0..T-1
     } else {
         e = make_tmap(&tB, a.xs, (uint64_t)a.H, (uint64_t)a.T * a.k, kBK, b_box);   // rows gathered in plan order
     }
@@ -920,21 +946,29 @@ GemmParams params(const ExpertArgs& a, bool up) {
 }
 
 // xs[pos] = x[perm[pos] / k]: token rows in plan order, one warp per row.
+// The rows are stored L2 evict-last: the up GEMM reads them next, once per
+// weight tile of their expert.
 __global__ void __launch_bounds__(256) k_gather_rows(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
                                                      uint16_t* __restrict__ xs, int P, int k, int H) {
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n16 = H / 8;
+    const uint64_t keep = policy_evict_last();
     for (int pos = blockIdx.x * 8 + warp; pos < P; pos += gridDim.x * 8) {
         const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)(perm[pos] / k) * H);
         uint4* dst = reinterpret_cast<uint4*>(xs + (size_t)pos * H);
-        for (int c = lane; c < n16; c += 32) dst[c] = ld_nc(src + c);
+        for (int c = lane; c < n16; c += 32) st_hint(dst + c, ld_nc(src + c), keep);
     }
     pdl_trigger();
 }
 
 }  // namespace
 
+
+// bf16 experts at T <= 16 tokens: every up tile multiplies all T token rows
+// of x (N = T rounded up to 16) and keeps the columns of the tokens routed to
+// its expert, so no rows are gathered into plan order first.
+bool gemm_up_reads_x(const ExpertArgs& a) { return a.fmt == 0 && a.T > 0 && a.T <= 16 && a.x != nullptr; }
 
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     const int P = a.T * a.k;
@@ -968,8 +1002,9 @@ cudaError_t gemm_down_q4(const ExpertArgs& a, const GemmParams& g, int bn, bool 
 }  // namespace
 
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    const GemmParams g = params(a, true);
+    GemmParams g = params(a, true);
     const int bn = pick_bn(a);
+    if (gemm_up_reads_x(a)) g.dense_n = (a.T + 15) & ~15;
     if (a.fmt == 0) {
         // token tiles of 128 and more: M = 256 tiles on SM pairs
         if (a.act == 0) {
@@ -998,6 +1033,20 @@ cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     if (a.fmt == 1) return gemm_down_q4<1>(a, g, bn, pdl, s);
     if (a.fmt == 2) return gemm_down_q4<2>(a, g, bn, pdl, s);
     return cudaErrorNotSupported;
+}
+
+cudaError_t make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* base,
+                         uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * elem_bytes};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 }  // namespace moe

@@ -447,12 +447,14 @@ cudaError_t q4_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_gemv_q4_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
+    if (gemv_q4t_fits(a, false)) return launch_gemv_q4t_up(a, pdl, s);
     if (a.fmt == kQAffine) return q4_up<kQAffine>(a, pdl, s);
     if (a.fmt == kQNvfp4) return q4_up<kQNvfp4>(a, pdl, s);
     return cudaErrorNotSupported;
 }
 
 cudaError_t launch_gemv_q4_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
+    if (gemv_q4t_fits(a, true)) return launch_gemv_q4t_down(a, pdl, s);
     if (a.fmt == kQAffine) return q4_down<kQAffine>(a, pdl, s);
     if (a.fmt == kQNvfp4) return q4_down<kQNvfp4>(a, pdl, s);
     return cudaErrorNotSupported;

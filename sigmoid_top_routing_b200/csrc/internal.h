@@ -91,6 +91,12 @@ cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // launch_gemv_up/down route fmt 1 and 2 here.
 cudaError_t launch_gemv_q4_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_q4_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
+// The TMA-fed 4-bit GEMV (gemv_q4t.cu), which launch_gemv_q4_up/down use
+// when gemv_q4t_fits: enough 128-row units for every SM and stage-aligned
+// scale rows.
+bool gemv_q4t_fits(const ExpertArgs& a, bool down);
+cudaError_t launch_gemv_q4t_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
+cudaError_t launch_gemv_q4t_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // MOE_DISPATCH_AUTO's choice: the GEMV for 4-bit experts with at most this
 // many routed pairs per expert on average, the tcgen05 GEMM otherwise.
 constexpr int kAffineGemvMaxPairsPerExpert = 8;
@@ -100,8 +106,10 @@ constexpr bool kNvfp4Gemm = true;
 cudaError_t launch_gemm_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemm_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // The up GEMM takes its token rows by TMA from xs, the rows of x in plan
-// order, filled by launch_gather_x before it.
+// order, filled by launch_gather_x before it -- except when
+// gemm_up_reads_x(a) (bf16 experts, T <= 16), where it reads x itself.
 cudaError_t launch_gather_x(const ExpertArgs& a, bool pdl, cudaStream_t s);
+bool gemm_up_reads_x(const ExpertArgs& a);
 cudaError_t launch_finalize(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // The one-expert identity plan of the shared expert: counts = {T},
 // offsets = {0, T}, perm = inv = 0..T-1, tiles = {0, ceil(T / 128)}, and

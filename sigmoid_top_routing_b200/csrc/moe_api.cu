@@ -298,7 +298,7 @@ struct Seq {
 moe_status run_experts(Seq& q, const ExpertArgs& a, const moe_dims* d, int dispatch) {
     const bool gemv = use_gemv(d, a.fmt, dispatch);
     cudaError_t e;
-    if (!gemv) {
+    if (!gemv && !gemm_up_reads_x(a)) {
         // token rows in plan order for the up GEMM's TMA (part of the plan's data movement)
         e = q.stage(MOE_STAGE_GATHER, [&](int*) { return launch_gather_x(a, true, q.s); });
         if (e != cudaSuccess) return cuda_fail(e, "gather token rows");

@@ -410,50 +410,67 @@ cudaError_t dispatch_select(const RouteArgs& a, bool fuse, bool pdl, cudaStream_
 // p_w[t][e]; k_select<.., PART> then forms L = p_0 + ... + p_7 in order, so
 // these logits are bit-identical to the one-CTA kernels', with 8x the CTAs.
 
-// T <= 32: CTA (expert e, segment w), one warp, lane = token; the next
-// chunk's token values and router row are loaded while this one is summed.
+// T <= 32: CTA (expert e, segment w), one warp, lane = token.  The
+// segment's router values and token rows (up to kSmallPass chunks at a time)
+// are requested by 16-byte cp.async all at once, so the loads pay one memory
+// latency rather than one per chunk; then each lane runs its chain from
+// shared memory.
+constexpr int kSmallPass = 8;                         // chunks staged per pass
+constexpr int kSmallRow = kSmallPass * kChunk + 8;    // bf16 per staged token row (+16 B: LDS.128 phases
+                                                      // of 8 lanes fall on distinct bank groups)
+
+MOE_DEV void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+
 __global__ void __launch_bounds__(32) k_logits_seg_small(RouteArgs a) {
+    __shared__ __align__(16) float s_w[kSmallPass * kChunk];
+    __shared__ __align__(16) uint16_t s_x[32 * kSmallRow];
     pdl_wait();
     zero_slice(a);
     const int e = blockIdx.x, w = blockIdx.y, lane = threadIdx.x;
-    const int H = a.H;
+    const int H = a.H, T = a.T;
     const int nch = (H / kChunk - w + kSegs - 1) / kSegs;
-    const bool tv = lane < a.T;
-    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(tv ? lane : 0) * H);
-    const float4* wr = reinterpret_cast<const float4*>(a.w_router + (size_t)e * H);
-    uint4 xv[4], xn[4];
-    float4 wv[8], wn[8];
-    auto load = [&](int j, uint4 (&xo)[4], float4 (&wo)[8]) {
-        const int h0 = (w + kSegs * j) * kChunk;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) xo[q] = ld_nc(xr + h0 / 8 + q);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) wo[q] = __ldg(wr + h0 / 4 + q);
-    };
+    const float* wr = a.w_router + (size_t)e * H;
     float acc = 0.0f;
-    if (nch > 0) load(0, xv, wv);
-    for (int j = 0; j < nch; ++j) {
-        if (j + 1 < nch) load(j + 1, xn, wn);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float4 w0 = wv[2 * q], w1 = wv[2 * q + 1];
-            acc = fmaf(bf16lo(xv[q].x), w0.x, acc);
-            acc = fmaf(bf16hi(xv[q].x), w0.y, acc);
-            acc = fmaf(bf16lo(xv[q].y), w0.z, acc);
-            acc = fmaf(bf16hi(xv[q].y), w0.w, acc);
-            acc = fmaf(bf16lo(xv[q].z), w1.x, acc);
-            acc = fmaf(bf16hi(xv[q].z), w1.y, acc);
-            acc = fmaf(bf16lo(xv[q].w), w1.z, acc);
-            acc = fmaf(bf16hi(xv[q].w), w1.w, acc);
+    for (int j0 = 0; j0 < nch; j0 += kSmallPass) {
+        const int np = min(kSmallPass, nch - j0);
+        // router: np chunks x 8 pieces of 16 B; tokens: T rows x np chunks x 4 pieces
+        for (int i = lane; i < np * 8; i += 32) {
+            const int j = i >> 3, q = i & 7;
+            cp_async16(s_w + j * kChunk + 4 * q, wr + (w + kSegs * (j0 + j)) * kChunk + 4 * q);
         }
-        if (j + 1 < nch) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) xv[q] = xn[q];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) wv[q] = wn[q];
+        for (int i = lane; i < T * np * 4; i += 32) {
+            const int t = i / (np * 4), r = i - t * np * 4, j = r >> 2, q = r & 3;
+            cp_async16(s_x + t * kSmallRow + j * kChunk + 8 * q,
+                       a.x + (size_t)t * H + (w + kSegs * (j0 + j)) * kChunk + 8 * q);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncwarp();
+        if (lane < T) {
+            const uint4* xr = reinterpret_cast<const uint4*>(s_x + lane * kSmallRow);
+            const float4* wv = reinterpret_cast<const float4*>(s_w);
+            for (int j = 0; j < np; ++j) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 xv = xr[j * 4 + q];
+                    const float4 w0 = wv[j * 8 + 2 * q], w1 = wv[j * 8 + 2 * q + 1];
+                    acc = fmaf(bf16lo(xv.x), w0.x, acc);
+                    acc = fmaf(bf16hi(xv.x), w0.y, acc);
+                    acc = fmaf(bf16lo(xv.y), w0.z, acc);
+                    acc = fmaf(bf16hi(xv.y), w0.w, acc);
+                    acc = fmaf(bf16lo(xv.z), w1.x, acc);
+                    acc = fmaf(bf16hi(xv.z), w1.y, acc);
+                    acc = fmaf(bf16lo(xv.w), w1.z, acc);
+                    acc = fmaf(bf16hi(xv.w), w1.w, acc);
+                }
+            }
+        }
+        __syncwarp();      // the next pass overwrites the staged values
     }
-    if (tv) a.part[((size_t)w * a.T + lane) * a.E + e] = acc;
+    if (lane < T) a.part[((size_t)w * T + lane) * a.E + e] = acc;
     pdl_trigger();
 }
 

@@ -33,10 +33,20 @@ def test_gemm_tiny(api):
     _check_all(inp, _gemm(api, inp))
 
 
-@pytest.mark.parametrize("T", [1, 8, 33])
+@pytest.mark.parametrize("T", [1, 8, 13, 16, 17, 33])
 def test_gemm_decode_shapes(api, T):
-    """Token tiles of width 32 (N = 16 or 32 per expert)."""
+    """Token tiles of width 32 (N = 16 or 32 per expert).  At T <= 16 the up
+    GEMM multiplies x itself (every token, N = T rounded up to 16) and keeps
+    the routed tokens' columns; above, it reads the rows gathered in plan
+    order."""
     inp = inputs_of(_small("lfm2_decode_t8", T))
+    _check_all(inp, _gemm(api, inp))
+
+
+@pytest.mark.parametrize("T", [5, 16])
+def test_gemm_relu2_x_operand(api, T):
+    """relu^2 up at T <= 16 (the x operand with its routed columns), E = 64, k = 6."""
+    inp = inputs_of(_small("nemotron_relu2_t2048", T))
     _check_all(inp, _gemm(api, inp))
 
 

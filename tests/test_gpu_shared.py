@@ -31,7 +31,8 @@ def _wl(base, T, shared_I, **over):
 
 @pytest.mark.parametrize("base,T,shared_I,dispatch", [
     ("nemotron_relu2_t2048", 300, 1536, None),   # tcgen05 GEMM, one expert, 300 tokens
-    ("lfm2_decode_t8", 8, 1792, None),           # 32-wide token tiles
+    ("lfm2_decode_t8", 8, 1792, None),           # 32-wide token tiles, the x operand (T <= 16)
+    ("nemotron_relu2_t2048", 12, 1536, None),    # relu^2, the x operand
     ("lfm2_decode_t8", 8, 1792, "gemv"),         # bf16 GEMV
     ("affine4_t8", 8, 1536, None),               # affine 4-bit register-dequant GEMV
 ])
