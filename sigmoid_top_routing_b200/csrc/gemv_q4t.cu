@@ -18,7 +18,7 @@
 // rows): for SwiGLU 64 features (their gate and up rows), else 128 rows.  A
 // stage is the unit's 128 rows x 512 k: four 64-row x 128-byte code boxes
 // (128-byte swizzle) and the rows' scales (NVFP4: 32 e4m3 bytes a row;
-// affine: 8 bf16 scales and 8 biases a row).  Each CTA (one per SM) takes a
+// affine: 8 bf16 scales and 8 biases a row).  Each CTA (one or two per SM) takes a
 // contiguous range of units in (expert, chunk, row block) order, so its
 // consecutive units share their token rows, which are staged in shared memory
 // only when the (expert, chunk) changes.  Eight consumer warps each own one
@@ -52,7 +52,6 @@ constexpr int kTW = 8;                                   // consumer warps
 constexpr int kTThreads = (kTW + 1) * 32;                // + the TMA producer warp
 constexpr int kTTok = 8;                                 // tokens per unit (the MMA's N)
 constexpr int kTStageK = 512;                            // k per stage
-constexpr int kTStages = 4;
 constexpr int kTBoxRows = 64;                            // rows per code box
 constexpr int kTCodeBox = kTBoxRows * 128;               // bytes of one code box (256 k x 64 rows)
 constexpr int kTCodeStage = 4 * kTCodeBox;               // [k half][row half] boxes
@@ -110,21 +109,22 @@ struct TLayout {          // dynamic shared memory of one CTA (byte offsets from
     int codes, scales, x, sx, bars, total;
 };
 
-MOE_DEV __host__ TLayout t_layout(int fmt, int K) {
+MOE_DEV __host__ TLayout t_layout(int fmt, int K, int stages) {
     TLayout L;
     L.codes = 0;
-    L.scales = L.codes + kTStages * kTCodeStage;
-    L.x = L.scales + kTStages * kTScaleStage;
+    L.scales = L.codes + stages * kTCodeStage;
+    L.x = L.scales + stages * kTScaleStage;
     int off = L.x + kTTok * t_xstride(K) * 2;
     L.sx = off;                                          // affine: sum_k x per (group, token), [G][8] fp32
     if (fmt == kTAffine) off += (t_kpad(K) / 64) * kTTok * 4;
     L.bars = (off + 7) & ~7;
-    L.total = L.bars + (2 * kTStages) * 8 + 1024;        // + alignment slack of the base
+    L.total = L.bars + (2 * stages) * 8 + 1024;          // + alignment slack of the base
     return L;
 }
 
-template <int FMT, int MODE>
-__global__ void __launch_bounds__(kTThreads, 1)
+// STG stages per CTA: 4 with one CTA per SM, 2 with two (the same bytes in flight per SM)
+template <int FMT, int MODE, int STG>
+__global__ void __launch_bounds__(kTThreads, 4 / STG)
     k_gemv_q4t(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmS,
                const __grid_constant__ CUtensorMap tmB, ExpertArgs a, uint32_t wait_limit) {
     extern __shared__ unsigned char t_smem_raw[];
@@ -138,16 +138,16 @@ __global__ void __launch_bounds__(kTThreads, 1)
     const int N = down ? a.H : (MODE == kTUpSwiglu ? 2 * a.I : a.I);    // weight rows per expert
     const int NRQ = MODE == kTUpSwiglu ? a.I / 64 : N / 128;             // units of rows per expert
     const int nst = t_kpad(K) / kTStageK;                               // stages per unit
-    const TLayout L = t_layout(FMT, K);
+    const TLayout L = t_layout(FMT, K, STG);
     const int XS = t_xstride(K);
     uint16_t* s_x = reinterpret_cast<uint16_t*>(sm + L.x);
     float* s_sx = reinterpret_cast<float*>(sm + L.sx);
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + L.bars);
-    uint64_t* empty = full + kTStages;
+    uint64_t* empty = full + STG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTStages; ++s) {
+        for (int s = 0; s < STG; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kTW);
         }
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                     }
                     used |= 1u << s;
                     par = (par & ~(1u << s)) | (ph << s);
-                    if (++s == kTStages) { s = 0; ph ^= 1; }
+                    if (++s == STG) { s = 0; ph ^= 1; }
                 }
             }
             if (!ok) {
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                 s_abort = 1;
             }
             // no copy of ours may still be in flight when the CTA exits
-            for (int q = 0; q < kTStages; ++q)
+            for (int q = 0; q < STG; ++q)
                 if (used & (1u << q)) mbar_wait(&full[q], (par >> q) & 1u, nullptr, wait_limit);
         }
     } else {
@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);   // this warp is done with the stage
-                if (++s == kTStages) { s = 0; ph ^= 1; }
+                if (++s == STG) { s = 0; ph ^= 1; }
             }
             if (dead) continue;
             // acc[0], acc[1]: MMA row g, tokens 2tq, 2tq + 1; acc[2], acc[3]: row g + 8
@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kTThreads, 1)
     pdl_trigger();
 }
 
-template <int FMT, int MODE>
+template <int FMT, int MODE, int STG>
 cudaError_t run_q4t(const ExpertArgs& a, int K, int N, bool pdl, cudaStream_t s) {
     const void* codes = MODE == kTDown ? a.w2 : a.w1;
     const void* scale = MODE == kTDown ? (const void*)a.w2_scale : (const void*)a.w1_scale;
@@ -502,11 +502,28 @@ cudaError_t run_q4t(const ExpertArgs& a, int K, int N, bool pdl, cudaStream_t s)
                              kTStageK / 64, kTBoxRows, false);
     }
     if (e != cudaSuccess) return e;
-    const TLayout L = t_layout(FMT, K);
-    auto kern = k_gemv_q4t<FMT, MODE>;
+    const TLayout L = t_layout(FMT, K, STG);
+    auto kern = k_gemv_q4t<FMT, MODE, STG>;
     if ((e = ensure_smem(kern, (size_t)L.total)) != cudaSuccess) return e;
-    return launch_k(kern, dim3(device_info().sm_count), dim3(kTThreads), (size_t)L.total, s, pdl, tC, tS, tB, a,
-                    sm100::kWaitLimit);
+    return launch_k(kern, dim3((4 / STG) * device_info().sm_count), dim3(kTThreads), (size_t)L.total, s, pdl, tC,
+                    tS, tB, a, sm100::kWaitLimit);
+}
+
+// Units of this projection (an estimate: about one chunk per active expert
+// plus one per 8 of the batch's pairs).
+long long q4t_units(const ExpertArgs& a, bool down) {
+    const int rows_unit = (!down && a.act == 0) ? 64 : 128;   // SwiGLU: 64 features (gate + up rows)
+    const int feats = down ? a.H : a.I;
+    const long long P = (long long)a.T * a.k;
+    const long long chunks = std::min<long long>(a.E, P) + P / kTTok;
+    return chunks * (feats / rows_unit);
+}
+
+// Two CTAs per SM (2 stages each) when there are >= 4 units per CTA, else one (4 stages).
+template <int FMT, int MODE>
+cudaError_t run_q4t_pick(const ExpertArgs& a, int K, int N, bool pdl, cudaStream_t s) {
+    if (q4t_units(a, MODE == kTDown) >= 8LL * device_info().sm_count) return run_q4t<FMT, MODE, 2>(a, K, N, pdl, s);
+    return run_q4t<FMT, MODE, 4>(a, K, N, pdl, s);
 }
 
 }  // namespace
@@ -517,32 +534,29 @@ cudaError_t run_q4t(const ExpertArgs& a, int K, int N, bool pdl, cudaStream_t s)
 bool gemv_q4t_fits(const ExpertArgs& a, bool down) {
     if (a.fmt != kTAffine && a.fmt != kTNvfp4) return false;
     const int K = down ? a.I : a.H;
-    const int rows_unit = (!down && a.act == 0) ? 64 : 128;   // SwiGLU: 64 features (gate + up rows)
+    const int rows_unit = (!down && a.act == 0) ? 64 : 128;
     const int feats = down ? a.H : a.I;
     if (feats % rows_unit) return false;
     if (a.fmt == kTNvfp4 ? (K % 256) : (K % 512)) return false;   // row strides of the scale tensors
-    if (t_layout(a.fmt, K).total + 4096 > device_info().max_smem_optin) return false;
-    // about as many (expert, chunk) units as the batch has chunks of its experts' tokens
-    const long long P = (long long)a.T * a.k;
-    const long long chunks = std::min<long long>(a.E, P) + P / kTTok;
-    return chunks * (feats / rows_unit) >= 4LL * device_info().sm_count;
+    if (t_layout(a.fmt, K, 4).total + 2048 > device_info().max_smem_optin) return false;
+    return q4t_units(a, down) >= 3LL * device_info().sm_count;      // >= 3 units per CTA at one CTA per SM
 }
 
 cudaError_t launch_gemv_q4t_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {
     if (a.fmt == kTAffine) {
-        if (a.act == 0) return run_q4t<kTAffine, kTUpSwiglu>(a, a.H, 2 * a.I, pdl, s);
-        return run_q4t<kTAffine, kTUpRelu2>(a, a.H, a.I, pdl, s);
+        if (a.act == 0) return run_q4t_pick<kTAffine, kTUpSwiglu>(a, a.H, 2 * a.I, pdl, s);
+        return run_q4t_pick<kTAffine, kTUpRelu2>(a, a.H, a.I, pdl, s);
     }
     if (a.fmt == kTNvfp4) {
-        if (a.act == 0) return run_q4t<kTNvfp4, kTUpSwiglu>(a, a.H, 2 * a.I, pdl, s);
-        return run_q4t<kTNvfp4, kTUpRelu2>(a, a.H, a.I, pdl, s);
+        if (a.act == 0) return run_q4t_pick<kTNvfp4, kTUpSwiglu>(a, a.H, 2 * a.I, pdl, s);
+        return run_q4t_pick<kTNvfp4, kTUpRelu2>(a, a.H, a.I, pdl, s);
     }
     return cudaErrorNotSupported;
 }
 
 cudaError_t launch_gemv_q4t_down(const ExpertArgs& a, bool pdl, cudaStream_t s) {
-    if (a.fmt == kTAffine) return run_q4t<kTAffine, kTDown>(a, a.I, a.H, pdl, s);
-    if (a.fmt == kTNvfp4) return run_q4t<kTNvfp4, kTDown>(a, a.I, a.H, pdl, s);
+    if (a.fmt == kTAffine) return run_q4t_pick<kTAffine, kTDown>(a, a.I, a.H, pdl, s);
+    if (a.fmt == kTNvfp4) return run_q4t_pick<kTNvfp4, kTDown>(a, a.I, a.H, pdl, s);
     return cudaErrorNotSupported;
 }
 
