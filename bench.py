@@ -19,7 +19,7 @@ dominant kernel (the expert up-projection), so the `roofline` entry is the
 average duration of the launches replayed inside the timed region, whatever K.
 
 The same process then measures the other configurations (`workloads` key: the
-decode block, the relu^2 block and the affine 4-bit token sweep), each with its
+decode block, the relu^2 block and the affine 4-bit and NVFP4 token sweeps), each with its
 own value, roofline and step roofline, on its own step count (about 0.3 s of
 work, at least 20 steps); the driver's K and W apply to the headline line.
 """
@@ -552,7 +552,10 @@ class Runner:
                 for _ in range(3):
                     g.replay()
             self.stream.synchronize()
-            out[nm] = round(1e3 * statistics.mean(a.elapsed_time(b) for a, b in evs), 2)
+            try:
+                out[nm] = round(1e3 * statistics.mean(a.elapsed_time(b) for a, b in evs), 2)
+            except RuntimeError:      # the stage launched no kernel of its own (events never recorded)
+                out[nm] = "not launched"
             del g
         return out
 
@@ -564,7 +567,7 @@ def dtype_of(wl) -> str:
 
 
 def gemv_path_of(wl, dispatch: str) -> bool:
-    """The library's AUTO choice: 4-bit experts at <= 8 pairs per expert take the GEMV."""
+    """The library's AUTO choice: 4-bit experts at <= 8 pairs per expert take a GEMV."""
     return dispatch == "gemv" or (dispatch == "auto" and wl.fmt != "bf16" and wl.T * wl.k <= 8 * wl.E
                                   and wl.H <= 8192 and wl.I <= 8192)
 

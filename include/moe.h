@@ -83,12 +83,12 @@ typedef enum { MOE_W_BF16 = 0, MOE_W_AFFINE4_G64 = 1, MOE_W_NVFP4 = 2 } moe_wfmt
 /* Which expert kernels run (per call through moe_exec_cfg, or the process-wide
  * default of moe_set_dispatch). */
 typedef enum {
-    MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM, except affine
-                              4-bit experts at <= 8 routed pairs per expert on average
-                              (T*k <= 8*E, H and I <= 8192), which take the
-                              register-dequant GEMV */
-    MOE_DISPATCH_GEMV = 1, /* the weight-streaming grouped GEMV (bf16: CUDA cores; affine
-                              4-bit: codes dequantised in registers, m16n8k16 dot products) */
+    MOE_DISPATCH_AUTO = 0, /* the library's choice: the tcgen05 grouped GEMM, except 4-bit
+                              (affine or NVFP4) experts at <= 8 routed pairs per expert on
+                              average (T*k <= 8*E, H and I <= 8192), which take the 4-bit GEMV */
+    MOE_DISPATCH_GEMV = 1, /* the weight-streaming grouped GEMV (bf16: CUDA cores; 4-bit: codes
+                              streamed by TMA or into registers and dequantised there,
+                              m16n8k16 dot products) */
     MOE_DISPATCH_GEMM = 2  /* the tcgen05 grouped GEMM */
 } moe_dispatch;
 

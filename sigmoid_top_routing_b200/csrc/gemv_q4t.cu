@@ -528,9 +528,8 @@ cudaError_t run_q4t_pick(const ExpertArgs& a, int K, int N, bool pdl, cudaStream
 
 }  // namespace
 
-// Whether the TMA-fed GEMV takes this projection: enough units for every SM
-// (a unit is <= 8 tokens x 128 weight rows), whole stages of code bytes and
-// scale rows that TMA can address, and the token tile within shared memory.
+// Whether the TMA-fed GEMV takes this projection: whole 128-row units, scale
+// rows that TMA can address, and the token tile within shared memory.
 bool gemv_q4t_fits(const ExpertArgs& a, bool down) {
     if (a.fmt != kTAffine && a.fmt != kTNvfp4) return false;
     const int K = down ? a.I : a.H;
@@ -538,8 +537,9 @@ bool gemv_q4t_fits(const ExpertArgs& a, bool down) {
     const int feats = down ? a.H : a.I;
     if (feats % rows_unit) return false;
     if (a.fmt == kTNvfp4 ? (K % 256) : (K % 512)) return false;   // row strides of the scale tensors
-    if (t_layout(a.fmt, K, 4).total + 2048 > device_info().max_smem_optin) return false;
-    return q4t_units(a, down) >= 3LL * device_info().sm_count;      // >= 3 units per CTA at one CTA per SM
+    // any unit count: with few units (one token) each busy SM still streams its
+    // units' codes with one pipeline ramp, where the register GEMV pays one per unit
+    return t_layout(a.fmt, K, 4).total + 2048 <= device_info().max_smem_optin;
 }
 
 cudaError_t launch_gemv_q4t_up(const ExpertArgs& a, bool pdl, cudaStream_t s) {

@@ -92,8 +92,8 @@ cudaError_t launch_gemv_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_q4_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_q4_down(const ExpertArgs& a, bool pdl, cudaStream_t s);
 // The TMA-fed 4-bit GEMV (gemv_q4t.cu), which launch_gemv_q4_up/down use
-// when gemv_q4t_fits: enough 128-row units for every SM and stage-aligned
-// scale rows.
+// when gemv_q4t_fits: whole 128-row units and stage-aligned scale rows; the
+// register GEMV takes the other shapes.
 bool gemv_q4t_fits(const ExpertArgs& a, bool down);
 cudaError_t launch_gemv_q4t_up(const ExpertArgs& a, bool pdl, cudaStream_t s);
 cudaError_t launch_gemv_q4t_down(const ExpertArgs& a, bool pdl, cudaStream_t s);

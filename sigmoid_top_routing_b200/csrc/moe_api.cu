@@ -216,8 +216,8 @@ moe_status check_route_args(const void* x, const float* logits, const float* w_r
 
 // bf16: the tcgen05 grouped GEMM serves every token count (its token tiles
 // shrink to 32 for decode batches); the CUDA-core GEMV stays selectable.
-// Affine 4-bit: up to a few pairs per expert the register-dequant GEMV streams
-// the codes faster than the GEMM's shared-memory dequant pipeline.
+// 4-bit (affine, NVFP4): up to a few pairs per expert the GEMVs stream the
+// codes faster than the GEMM's shared-memory dequant pipeline.
 bool use_gemv(const moe_dims* d, int32_t fmt, int mode) {
     if (mode != MOE_DISPATCH_AUTO) return mode == MOE_DISPATCH_GEMV;
     if (fmt == MOE_W_NVFP4 && !kNvfp4Gemm) return true;   // no tcgen05 NVFP4 path in this build

@@ -63,10 +63,27 @@ def test_affine4_gemv_relu2(api):
     _check_all(inp, run_forward(api, inp, dispatch=abi.MOE_DISPATCH_GEMV))
 
 
-def test_affine4_t512(api):
-    """Token tiles of 128: two accumulators (gate, up) per SwiGLU tile."""
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+def test_affine4_t512(api, path):
+    """32 pairs per expert: AUTO runs the tcgen05 path (token tiles of 128,
+    interleaved SwiGLU tiles); the TMA GEMV is forced (four 8-token chunks per
+    expert on average, the hot experts' many more)."""
+    from sigmoid_top_routing_b200 import abi
+    d = {"auto": abi.MOE_DISPATCH_AUTO, "gemv": abi.MOE_DISPATCH_GEMV}[path]
     inp = inputs_of(G.WORKLOADS["affine4_t512"])
-    _check_all(inp, run_forward(api, inp))
+    _check_all(inp, run_forward(api, inp, dispatch=d))
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_affine4_tma_gemv_many_chunks(api, act):
+    """The TMA GEMV (forced) at 48 pairs per expert on average: six 8-token
+    chunks per expert, ragged, H = 1024 (two stages of K), I = 512, 2 all-NaN
+    token rows."""
+    from sigmoid_top_routing_b200 import abi
+    wl = G.Workload("a4_mid", T=96, H=1024, E=8, k=4, I=512, act=act, fmt="affine4", nan_rows=2)
+    inp = inputs_of(wl)
+    rep = _check_all(inp, run_forward(api, inp, dispatch=abi.MOE_DISPATCH_GEMV))
+    assert rep.nan_rows == 2
 
 
 def test_affine4_t8192_full(api):

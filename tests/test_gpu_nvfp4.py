@@ -44,9 +44,25 @@ def test_nvfp4_decode_sizes(api, T):
     _check_all(inp, run_forward(api, inp))
 
 
-def test_nvfp4_t512(api):
+@pytest.mark.parametrize("path", ["auto", "gemv"])
+def test_nvfp4_t512(api, path):
+    """AUTO: the tcgen05 path; forced: the TMA GEMV over many 8-token chunks."""
+    from sigmoid_top_routing_b200 import abi
+    d = {"auto": abi.MOE_DISPATCH_AUTO, "gemv": abi.MOE_DISPATCH_GEMV}[path]
     inp = inputs_of(G.WORKLOADS["nvfp4_t512"])
-    _check_all(inp, run_forward(api, inp))
+    _check_all(inp, run_forward(api, inp, dispatch=d))
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu2"])
+def test_nvfp4_tma_gemv_many_chunks(api, act):
+    """The TMA GEMV (forced) at 48 pairs per expert: six 8-token chunks per
+    expert, H = 1024, I = 512 (K of the down projection: one stage), 2 all-NaN
+    token rows."""
+    from sigmoid_top_routing_b200 import abi
+    wl = G.Workload("n4_mid", T=96, H=1024, E=8, k=4, I=512, act=act, fmt="nvfp4", nan_rows=2)
+    inp = inputs_of(wl)
+    rep = _check_all(inp, run_forward(api, inp, dispatch=abi.MOE_DISPATCH_GEMV))
+    assert rep.nan_rows == 2
 
 
 def test_nvfp4_t8192_full(api):

@@ -49,7 +49,7 @@ def test_bf16_gemv(api):
 
 @pytest.mark.parametrize("T", [8, 512])
 def test_affine4(api, T):
-    """T = 8 runs the register-dequant GEMV, T = 512 the tcgen05 GEMM."""
+    """T = 8 runs the TMA-fed 4-bit GEMV, T = 512 the tcgen05 GEMM."""
     inp = inputs_of(G.WORKLOADS[f"affine4_t{T}"])
     _check_all(inp, run_forward(api, inp))
 

@@ -34,7 +34,7 @@ def _wl(base, T, shared_I, **over):
     ("lfm2_decode_t8", 8, 1792, None),           # 32-wide token tiles, the x operand (T <= 16)
     ("nemotron_relu2_t2048", 12, 1536, None),    # relu^2, the x operand
     ("lfm2_decode_t8", 8, 1792, "gemv"),         # bf16 GEMV
-    ("affine4_t8", 8, 1536, None),               # affine 4-bit register-dequant GEMV
+    ("affine4_t8", 8, 1536, None),               # affine 4-bit TMA-fed GEMV
 ])
 def test_shared_expert_alone(api, base, T, shared_I, dispatch):
     import oracle as O

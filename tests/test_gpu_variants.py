@@ -57,7 +57,7 @@ def test_nemotron_eps(api):
     ("lfm2_decode_t8", 8, None),          # tcgen05 GEMM, 32-wide tiles (gate and up halves in one tile)
     ("lfm2_prefill_t4096", 600, None),    # 128-wide tiles, two accumulators
     ("lfm2_decode_t8", 17, "gemv"),       # bf16 CUDA-core GEMV
-    ("affine4_t8", 8, None),              # affine 4-bit register-dequant GEMV
+    ("affine4_t8", 8, None),              # affine 4-bit TMA-fed GEMV
     ("affine4_t512", 512, None),          # affine 4-bit tcgen05 GEMM
 ])
 def test_swiglu_limit(api, base, T, dispatch):
