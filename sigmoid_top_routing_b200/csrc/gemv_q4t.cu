@@ -519,10 +519,14 @@ long long q4t_units(const ExpertArgs& a, bool down) {
     return chunks * (feats / rows_unit);
 }
 
-// Two CTAs per SM (2 stages each) when there are >= 4 units per CTA, else one (4 stages).
+// Two CTAs per SM (2 stages each) when there are >= 4 units per CTA and both fit, else one (4 stages).
 template <int FMT, int MODE>
 cudaError_t run_q4t_pick(const ExpertArgs& a, int K, int N, bool pdl, cudaStream_t s) {
-    if (q4t_units(a, MODE == kTDown) >= 8LL * device_info().sm_count) return run_q4t<FMT, MODE, 2>(a, K, N, pdl, s);
+    // (two CTAs only when both fit in one SM's shared memory with their static
+    // arrays and the 1 KB the hardware reserves per CTA)
+    const DeviceInfo& di = device_info();
+    const bool two_fit = 2 * (t_layout(FMT, K, 2).total + 2048 + 1024) <= di.smem_per_sm;
+    if (two_fit && q4t_units(a, MODE == kTDown) >= 8LL * di.sm_count) return run_q4t<FMT, MODE, 2>(a, K, N, pdl, s);
     return run_q4t<FMT, MODE, 4>(a, K, N, pdl, s);
 }
 

@@ -73,7 +73,8 @@ struct ExpertArgs {
 
 struct DeviceInfo {
     int sm_count;
-    int max_smem_optin;
+    int max_smem_optin;      // dynamic shared memory one CTA may opt into
+    int smem_per_sm;         // shared memory of one SM (all resident CTAs together)
     int* err_word;           // device address of this device's error word
 };
 

@@ -26,6 +26,7 @@ const DeviceInfo& device_info() {
     DeviceInfo di{};
     cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev);
     cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaDeviceGetAttribute(&di.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.err_word), g_err_word) != cudaSuccess)
         di.err_word = nullptr;
     if (di.sm_count <= 0) di.sm_count = 1;
